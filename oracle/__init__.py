@@ -1,0 +1,31 @@
+"""CPU oracle for the fused rotate + quantize operator (test infrastructure).
+
+This package is test infrastructure only. It is imported by `tests/`, by
+`__graft_entry__.smoke()` and by the `cpu_baseline` / `--impl reference` legs of
+`bench.py`, and by nothing else. The product path (the CUDA library and its
+Python binding) never imports, links or executes it, and the two share no code.
+
+Source: "aclnnFlatQuantV2 complete guide: from two-level matmul to FP4 E2M1
+quantization fusion" (http://www.zwxr.cn/news/277566), sections "How it works",
+"per-token mode", "per-group mode" cases 1-3, "Parameter quick reference" and
+"Error code quick reference".
+
+Parity unpinned: none. Every public function here is pinned by
+`tests/test_oracle_pins.py` against closed forms, brute force, hand-worked values
+or textbook special cases.
+"""
+
+from .flatquant import (  # noqa: F401
+    E2M1_GRID,
+    e2m1_encode,
+    e2m1_decode,
+    rotate,
+    per_token_quantize,
+    pack_nibbles,
+    mx_group_view,
+    mx_scale_exponent,
+    mx_quantize,
+    mx_scale_layout,
+    flat_quant_per_token,
+    flat_quant_mx,
+)
