@@ -1,0 +1,209 @@
+"""Python binding of libfq: the C ABI calls with torch tensors for device memory.
+
+Every step of the operator runs in libfq's CUDA kernels; this module only checks
+tensor placement, allocates outputs with torch, and passes pointers and the current
+CUDA stream. There is no CPU implementation here.
+"""
+
+import ctypes
+
+import torch
+
+from . import _lib
+
+_DT = {torch.bfloat16: _lib.FQ_BF16, torch.float16: _lib.FQ_FP16}
+
+
+def _stream_ptr(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _check_input(name, t, dtype=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (libfq has no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must have dtype {dtype}, got {t.dtype}")
+
+
+class FlatQuant:
+    """A plan for one shape [K, M, N] and input dtype (the handle of fq_create)."""
+
+    def __init__(self, K, M, N, dtype=torch.bfloat16, kernel="auto"):
+        lib = _lib.load()
+        if dtype not in _DT:
+            raise ValueError("dtype must be torch.bfloat16 or torch.float16")
+        self.K, self.M, self.N, self.dtype = int(K), int(M), int(N), dtype
+        h = ctypes.c_void_p()
+        _lib.check(lib.fq_create(ctypes.byref(h), self.K, self.M, self.N, _DT[dtype]),
+                   "fq_create")
+        self._h = h
+        self._lib = lib
+        self.set_kernel(kernel)
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            self._lib.fq_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def set_kernel(self, kernel):
+        code = {"auto": _lib.FQ_KERNEL_AUTO, "general": _lib.FQ_KERNEL_GENERAL,
+                "tcgen05": _lib.FQ_KERNEL_TCGEN05}[kernel]
+        _lib.check(self._lib.fq_set_kernel(self._h, code), "fq_set_kernel")
+
+    @property
+    def last_kernel(self):
+        return {0: "auto", 1: "general", 2: "tcgen05"}[self._lib.fq_last_kernel(self._h)]
+
+    @property
+    def last_launch_count(self):
+        return self._lib.fq_last_launch_count(self._h)
+
+    def device_status(self):
+        v = ctypes.c_uint32(0)
+        st = self._lib.fq_device_status(self._h, ctypes.byref(v))
+        if st not in (_lib.FQ_OK, _lib.FQ_ERR_DEVICE_TIMEOUT):
+            _lib.check(st, "fq_device_status")
+        return int(v.value)
+
+    def _inputs(self, x, P1, P2, allow_no_p2=False):
+        _check_input("x", x, self.dtype)
+        _check_input("P1", P1, self.dtype)
+        if tuple(x.shape) != (self.K, self.M, self.N):
+            raise ValueError(f"x must have shape {(self.K, self.M, self.N)}, got {tuple(x.shape)}")
+        if tuple(P1.shape) != (self.M, self.M):
+            raise ValueError("P1 must be [M, M]")
+        if P2 is not None and P2.numel() == 0 and allow_no_p2:
+            P2 = None
+        if P2 is None:
+            if not allow_no_p2:
+                raise ValueError("P2 is required in per-token mode")
+        else:
+            _check_input("P2", P2, self.dtype)
+            if tuple(P2.shape) != (self.N, self.N):
+                raise ValueError("P2 must be [N, N]")
+        return P2
+
+    def quantize_per_token(self, x, P1, P2, clip_ratio=1.0, out_dtype="int4",
+                           out=None, quant_scale=None, stream=None):
+        """Per-token INT4 quantization of P1 . (x . P2). Returns (out, quantScale):
+        out is uint8 [K, M*N/2] for "int4" or int32 [K, M, N/8] for "int32"."""
+        self._inputs(x, P1, P2)
+        K, M, N = self.K, self.M, self.N
+        if out is None:
+            if out_dtype == "int32":
+                out = torch.empty((K, M, N // 8), dtype=torch.int32, device=x.device)
+            else:
+                out = torch.empty((K, M * N // 2), dtype=torch.uint8, device=x.device)
+        if quant_scale is None:
+            quant_scale = torch.empty((K,), dtype=torch.float32, device=x.device)
+        fmt = _lib.FQ_OUT_INT32 if out_dtype == "int32" else _lib.FQ_OUT_INT4
+        _lib.check(self._lib.fq_quantize_per_token(
+            self._h, _ptr(x), _ptr(P1), _ptr(P2), float(clip_ratio), fmt, _ptr(out),
+            _ptr(quant_scale), _stream_ptr(stream)), "fq_quantize_per_token")
+        return out, quant_scale
+
+    def quantize_mx(self, x, P1, P2, dst_type_max=0.0, out=None, scales=None, stream=None):
+        """Per-group E2M1 + E8M0 quantization of P1 . (x . P2) (P2 None skips the right
+        multiply). Returns (out uint8 [K, M*N/2], scales uint8 [K, ceilDiv(M*N,64), 2])."""
+        P2 = self._inputs(x, P1, P2, allow_no_p2=True)
+        K, M, N = self.K, self.M, self.N
+        if out is None:
+            out = torch.empty((K, M * N // 2), dtype=torch.uint8, device=x.device)
+        if scales is None:
+            scales = torch.empty((K, -(-M * N // 64), 2), dtype=torch.uint8, device=x.device)
+        _lib.check(self._lib.fq_quantize_mx(
+            self._h, _ptr(x), _ptr(P1), _ptr(P2), float(dst_type_max), _ptr(out),
+            _ptr(scales), _stream_ptr(stream)), "fq_quantize_mx")
+        return out, scales
+
+    def debug_rotate(self, x, P1, P2, out=None, stream=None):
+        """x'' = P1 . (x . P2) as float32 [K, M, N] (test hook)."""
+        P2 = self._inputs(x, P1, P2, allow_no_p2=True)
+        if out is None:
+            out = torch.empty((self.K, self.M, self.N), dtype=torch.float32, device=x.device)
+        _lib.check(self._lib.fq_debug_rotate(self._h, _ptr(x), _ptr(P1), _ptr(P2), _ptr(out),
+                                             _stream_ptr(stream)), "fq_debug_rotate")
+        return out
+
+
+def quantize_per_token(x, P1, P2, clip_ratio=1.0, out_dtype="int4", kernel="auto"):
+    K, M, N = x.shape
+    return FlatQuant(K, M, N, x.dtype, kernel).quantize_per_token(x, P1, P2, clip_ratio, out_dtype)
+
+
+def quantize_mx(x, P1, P2, dst_type_max=0.0, kernel="auto"):
+    K, M, N = x.shape
+    return FlatQuant(K, M, N, x.dtype, kernel).quantize_mx(x, P1, P2, dst_type_max)
+
+
+def debug_rotate(x, P1, P2, kernel="auto"):
+    K, M, N = x.shape
+    return FlatQuant(K, M, N, x.dtype, kernel).debug_rotate(x, P1, P2)
+
+
+class HostPipeline:
+    """End-to-end use from host memory: pinned host inputs are copied to device staging
+    buffers, the operator runs, and the packed outputs and scales are copied back, all on
+    one stream. The device buffers are allocated once, in the constructor."""
+
+    def __init__(self, fq: FlatQuant, mode, out_dtype="int4", device=None):
+        self.fq = fq
+        self.mode = mode
+        self.out_dtype = out_dtype
+        dev = device or torch.device("cuda", torch.cuda.current_device())
+        K, M, N = fq.K, fq.M, fq.N
+        self.x = torch.empty((K, M, N), dtype=fq.dtype, device=dev)
+        self.P1 = torch.empty((M, M), dtype=fq.dtype, device=dev)
+        self.P2 = torch.empty((N, N), dtype=fq.dtype, device=dev)
+        if mode == "per_token":
+            if out_dtype == "int32":
+                self.out = torch.empty((K, M, N // 8), dtype=torch.int32, device=dev)
+            else:
+                self.out = torch.empty((K, M * N // 2), dtype=torch.uint8, device=dev)
+            self.scale = torch.empty((K,), dtype=torch.float32, device=dev)
+        else:
+            self.out = torch.empty((K, M * N // 2), dtype=torch.uint8, device=dev)
+            self.scale = torch.empty((K, -(-M * N // 64), 2), dtype=torch.uint8, device=dev)
+
+    def host_outputs(self):
+        """Pinned host buffers shaped like the outputs."""
+        return (torch.empty_like(self.out, device="cpu").pin_memory(),
+                torch.empty_like(self.scale, device="cpu").pin_memory())
+
+    def h2d_bytes(self):
+        return sum(t.numel() * t.element_size() for t in (self.x, self.P1, self.P2))
+
+    def d2h_bytes(self):
+        return sum(t.numel() * t.element_size() for t in (self.out, self.scale))
+
+    def run(self, x_host, P1_host, P2_host, out_host, scale_host, clip_ratio=1.0,
+            dst_type_max=0.0, stream=None):
+        s = stream if stream is not None else torch.cuda.current_stream()
+        with torch.cuda.stream(s):
+            self.x.copy_(x_host, non_blocking=True)
+            self.P1.copy_(P1_host, non_blocking=True)
+            self.P2.copy_(P2_host, non_blocking=True)
+            if self.mode == "per_token":
+                self.fq.quantize_per_token(self.x, self.P1, self.P2, clip_ratio, self.out_dtype,
+                                           out=self.out, quant_scale=self.scale, stream=s)
+            else:
+                self.fq.quantize_mx(self.x, self.P1, self.P2, dst_type_max, out=self.out,
+                                    scales=self.scale, stream=s)
+            out_host.copy_(self.out, non_blocking=True)
+            scale_host.copy_(self.scale, non_blocking=True)
+        return out_host, scale_host

@@ -1,0 +1,53 @@
+// Internal declarations shared by the host layer and the kernels of libfq.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "fq_quant.cuh"
+
+namespace fq {
+
+enum Mode : int { kModePerToken = 0, kModeMx = 1, kModeRotate = 2 };
+
+struct GeneralParams {
+  const void* x;       // [K, M, N] 16-bit
+  const void* P1;      // [M, M]
+  const void* P2;      // [N, N] or nullptr (skip the right multiply)
+  int64_t K;
+  int M, N;
+  int mode;            // Mode
+  double clip_ratio;   // per-token
+  MxRule rule;         // per-group
+  uint8_t* out;        // packed codes, K*M*N/2 bytes
+  float* quant_scale;  // [K] per-token
+  uint8_t* scales;     // [K, 2*ceilDiv(M*N,64)] per-group
+  float* x2;           // [K, M, N] rotate-only
+};
+
+size_t general_smem_bytes(int M, int N, int elem_bytes);
+cudaError_t launch_general(const GeneralParams& p, bool fp16_in, int grid, cudaStream_t stream);
+
+// Tensor-core kernel: M in {32, 64, 128} (128/M tokens per 128-row tile), N a multiple
+// of 16 in [64, 128], 16-byte aligned x / out / scales, M*N a multiple of 32.
+struct TcParams {
+  const void* x;
+  const void* P1;
+  const void* P2;      // nullptr: identity right multiply
+  int64_t K;
+  int M, N;
+  int mode;
+  double clip_ratio;
+  MxRule rule;
+  uint8_t* out;
+  float* quant_scale;
+  uint8_t* scales;
+  float* x2;
+  uint32_t* status;    // device status word (bounded waits)
+};
+
+bool tc_supported(int64_t K, int M, int N);
+cudaError_t launch_tc(const TcParams& p, bool fp16_in, int num_sms, cudaStream_t stream);
+
+}  // namespace fq

@@ -1,0 +1,141 @@
+"""Comparison of the CUDA outputs with the oracle under the stated tolerance.
+
+Tolerance (bit-exact on codes and scale exponents, except near rounding boundaries):
+  * an element is exempt when the oracle's value before rounding lies within 1e-5
+    (relative) of a rounding boundary: k + 0.5 for INT4, the E2M1 midpoints 0.25, 0.75,
+    1.25, 1.75, 2.5, 3.5, 5 for E2M1;
+  * a group is exempt when its oracle absmax lies within 1e-5 (relative) of an exponent
+    boundary of its rule (a power of two; for 6.0 / 7.0 also 1.5 / 1.75 times one; for
+    the ratio rule, amax / dstTypeMax near a power of two);
+  * exempt elements may differ by one code step, exempt groups by one exponent step (and
+    then their codes are not compared); at most 0.01% of elements may differ at all.
+  * the per-token float32 quantScale is compared to a relative 1e-6 (its only source of
+    difference is the float32 rounding of x'' inside the kernel).
+"""
+
+import numpy as np
+
+REL = 1e-5
+MAX_MISMATCH_FRAC = 1e-4
+E2M1_MIDS = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+E2M1_MAG = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def unpack_nibbles(b):
+    b = np.asarray(b, dtype=np.uint8)
+    out = np.empty(b.shape[:-1] + (b.shape[-1] * 2,), dtype=np.uint8)
+    out[..., 0::2] = b & 0xF
+    out[..., 1::2] = b >> 4
+    return out
+
+
+def int4_exempt(v):
+    v = np.asarray(v, dtype=np.float64)
+    b = np.floor(v) + 0.5
+    return np.abs(v - b) <= REL * np.abs(b)
+
+
+def e2m1_exempt(v):
+    a = np.abs(np.asarray(v, dtype=np.float64))
+    d = np.abs(a[..., None] - E2M1_MIDS)
+    return np.any(d <= REL * E2M1_MIDS, axis=-1)
+
+
+def _near_pow2(a):
+    a = np.asarray(a, dtype=np.float64)
+    pos = a > 0
+    s = np.where(pos, a, 1.0)
+    m = s / np.exp2(np.floor(np.log2(s)))
+    return pos & ((m <= 1 + REL) | (m >= 2 * (1 - REL)))
+
+
+def group_exempt(amax, D):
+    amax = np.asarray(amax, dtype=np.float64)
+    if D == 0.0:
+        return _near_pow2(amax)
+    if D in (6.0, 7.0):
+        pos = amax > 0
+        s = np.where(pos, amax, 1.0)
+        m = s / np.exp2(np.floor(np.log2(s)))
+        t = D / 4.0
+        return _near_pow2(amax) | (pos & (np.abs(m - t) <= REL * t))
+    return _near_pow2(amax / D)
+
+
+def compare_per_token(out_bytes, qs, ref_codes, ref_qs, ref_v):
+    """out_bytes: uint8 [K, M*N/2] from the GPU; ref_* from oracle.per_token_quantize."""
+    K = ref_codes.shape[0]
+    got = unpack_nibbles(np.asarray(out_bytes).reshape(K, -1)).astype(np.int64)
+    got = np.where(got >= 8, got - 16, got)
+    want = ref_codes.reshape(K, -1).astype(np.int64)
+    v = ref_v.reshape(K, -1)
+    diff = got != want
+    exempt = int4_exempt(v)
+    stats = {"elements": int(want.size), "mismatch": int(diff.sum()),
+             "exempt_mismatch": int((diff & exempt).sum())}
+    bad = diff & ~exempt
+    assert not bad.any(), f"non-exempt INT4 mismatches: {int(bad.sum())} {stats}"
+    assert np.all(np.abs(got - want)[diff] <= 1), "exempt INT4 codes differ by more than one"
+    assert stats["mismatch"] <= MAX_MISMATCH_FRAC * want.size, stats
+    qs = np.asarray(qs, dtype=np.float64)
+    rq = np.asarray(ref_qs, dtype=np.float64)
+    rel = np.abs(qs - rq) / np.maximum(np.abs(rq), 1e-30)
+    stats["quant_scale_max_rel"] = float(rel.max()) if rel.size else 0.0
+    assert np.all(rel <= 1e-6), f"quantScale differs: max rel {rel.max()}"
+    return stats
+
+
+def _e2m1_step(a_codes, b_codes):
+    """Distance in code steps between two E2M1 codes on the signed number line."""
+    def pos(c):
+        mag = (c & 7).astype(np.int64)
+        return np.where(c & 8, -mag, mag)
+    return np.abs(pos(a_codes) - pos(b_codes))
+
+
+def compare_mx(out_bytes, scales, ref_info, D):
+    """out_bytes uint8 [K, M*N/2], scales uint8 [K, S, 2] from the GPU; ref_info from
+    oracle.flat_quant_mx."""
+    ref_codes = ref_info["codes"]
+    K, L = ref_codes.shape
+    G = ref_info["group_bytes"].shape[1]
+    got = unpack_nibbles(np.asarray(out_bytes).reshape(K, -1))[:, :L]
+    got_b = np.asarray(scales).reshape(K, -1)
+    want_b = ref_info["group_bytes"]
+    # the pad slot of an odd group count is 0x00
+    if got_b.shape[1] > G:
+        assert np.all(got_b[:, G:] == 0), "pad scale byte is not 0x00"
+    got_b = got_b[:, :G].astype(np.int64)
+    gex = group_exempt(ref_info["amax"], D)
+    bdiff = got_b != want_b.astype(np.int64)
+    assert not (bdiff & ~gex).any(), \
+        f"non-exempt E8M0 mismatches: {int((bdiff & ~gex).sum())}"
+    assert np.all(np.abs(got_b - want_b)[bdiff] <= 1)
+    # element codes, skipping groups whose exponent legitimately differs
+    skip = np.repeat(bdiff, 32, axis=1)[:, :L]
+    v = ref_info["v"].reshape(K, -1)[:, :L]
+    diff = (got != ref_codes) & ~skip
+    exempt = e2m1_exempt(v) | np.repeat(gex, 32, axis=1)[:, :L]
+    bad = diff & ~exempt
+    stats = {"elements": int(ref_codes.size), "groups": int(K * G),
+             "scale_mismatch": int(bdiff.sum()), "mismatch": int(diff.sum()),
+             "exempt_mismatch": int((diff & exempt).sum())}
+    assert not bad.any(), f"non-exempt E2M1 mismatches: {int(bad.sum())} {stats}"
+    assert np.all(_e2m1_step(got[diff], ref_codes[diff]) <= 1), "exempt E2M1 codes differ by more than one step"
+    total = stats["mismatch"] + 32 * stats["scale_mismatch"]
+    assert total <= MAX_MISMATCH_FRAC * ref_codes.size, stats
+    return stats
+
+
+def rotate_close(x2_gpu, x2_ref):
+    """x'' within 2e-3 relative: |d| <= 2e-3 * max(|ref|, 1e-3 * amax_token). Returns the
+    largest error divided by the token's rms (a finer figure that is reported)."""
+    K = x2_ref.shape[0]
+    g = np.asarray(x2_gpu, dtype=np.float64).reshape(K, -1)
+    r = np.asarray(x2_ref, dtype=np.float64).reshape(K, -1)
+    amax = np.abs(r).max(axis=1, keepdims=True)
+    tol = 2e-3 * np.maximum(np.abs(r), 1e-3 * amax)
+    d = np.abs(g - r)
+    assert np.all(d <= tol), f"x'' outside tolerance: worst {float((d / np.maximum(tol, 1e-300)).max())}"
+    rms = np.sqrt((r * r).mean(axis=1, keepdims=True))
+    return float((d / np.maximum(rms, 1e-300)).max())
