@@ -33,9 +33,10 @@ Readings taken where the page is silent or garbled (each is listed in the design doc)
 * Case 2 reads the mantissa check as "the significand's leading one (6.0) or two
   (7.0) fraction bits are 1 and the remaining fraction bits are not all zero", in
   which case the exponent is rounded up.
-* E2M1 casts round to nearest with ties to the even code and saturate to +-6; a
-  nonzero negative value keeps its sign bit even when it rounds to zero; an
-  exactly-zero value encodes as 0x0.
+* E2M1 casts round to nearest with ties to the even code and saturate to +-6; every
+  value whose magnitude rounds to zero encodes as +0 (0x0), so the format's two zero
+  codes never both appear (the page gives no rule for the sign of a zero code, and a
+  sign kept on values that round to zero would hinge on the last bit of x'').
 * The pad byte of an odd group count is the scale of a group of 32 zeros (0x00).
 """
 
@@ -50,7 +51,7 @@ GROUP = 32  # per-group mode: 32 consecutive elements share one E8M0 exponent
 def e2m1_encode(v):
     """E2M1 cast of float values (page: per-group mode, "P_i = cast_to_dst_type(V_i /
     mxscale, round_mode)"): nearest grid magnitude, ties to the even code, values above
-    6 saturate to 6, sign in bit 3. Returns uint8 codes in [0, 15].
+    6 saturate to 6, sign in bit 3 for nonzero magnitudes. Returns uint8 codes in [0, 15].
 
     Brute force: every value is compared with all eight grid magnitudes."""
     v = np.asarray(v, dtype=np.float64)
@@ -59,7 +60,7 @@ def e2m1_encode(v):
     nearest = dist == dist.min(axis=-1, keepdims=True)
     even_bonus = 2 - (np.arange(8) % 2)  # even codes win ties
     mag = np.argmax(nearest * even_bonus, axis=-1).astype(np.uint8)
-    neg = (v < 0).astype(np.uint8)  # -0.0 and +0.0 both count as not negative
+    neg = ((v < 0) & (mag > 0)).astype(np.uint8)  # a zero magnitude is always +0 (0x0)
     return mag | (neg << 3)
 
 

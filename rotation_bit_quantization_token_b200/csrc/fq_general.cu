@@ -120,7 +120,7 @@ general_kernel(const GeneralParams p) {
             if (valid && (c & 1) == 0) {
               uint32_t byte;
               if (p.mode == kModePerToken) byte = int4_nibble(v) | (int4_nibble(v_hi) << 4);
-              else byte = e2m1x2(v, v_hi);
+              else byte = e2m1_canonical_zero(e2m1x2_raw(v, v_hi));
               p.out[(k * MN + f) >> 1] = uint8_t(byte);
             }
           }

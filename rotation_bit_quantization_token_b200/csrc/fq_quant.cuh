@@ -67,11 +67,9 @@ __device__ __forceinline__ MxScale mx_scale(float amax, MxRule rule) {
 }
 
 // Two E2M1 codes (round to nearest even, saturate to +-6) packed in one byte: `lo` in
-// bits 0-3, `hi` in bits 4-7. An exactly-zero input encodes as +0 (0x0); nonzero
-// negative values keep the sign bit even when they round to zero.
-__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
-  lo = __fadd_rn(lo, 0.0f);  // -0.0 -> +0.0, every other value unchanged
-  hi = __fadd_rn(hi, 0.0f);
+// bits 0-3, `hi` in bits 4-7. The hardware conversion keeps the sign of values that round
+// to zero; e2m1_canonical_zero() removes it.
+__device__ __forceinline__ uint32_t e2m1x2_raw(float lo, float hi) {
   uint16_t r;
   // The first source operand lands in the upper nibble, the second in the lower.
   asm("{\n\t.reg .b8 t;\n\t"
@@ -80,6 +78,14 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
       : "=h"(r)
       : "f"(hi), "f"(lo));
   return uint32_t(r) & 0xFFu;
+}
+
+// Clears the sign bit of every E2M1 nibble whose magnitude is zero (eight nibbles per
+// word): a zero code is always +0 (0x0). For a nibble n, (n & 7) + 7 sets bit 3 exactly
+// when the magnitude is nonzero, with no carry into the next nibble.
+__device__ __forceinline__ uint32_t e2m1_canonical_zero(uint32_t w) {
+  const uint32_t nonzero = ((w & 0x77777777u) + 0x77777777u) & 0x88888888u;
+  return w & (0x77777777u | nonzero);
 }
 
 // INT4 code: round half to even, clamp to [-8, 7], as a 4-bit two's complement nibble.

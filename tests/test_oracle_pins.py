@@ -188,7 +188,7 @@ def _e2m1_by_scaling(v):
     step = np.where(a < 2, 0.5, np.where(a < 4, 1.0, 2.0))
     q = np.minimum(np.rint(a / step) * step, 6.0)
     idx = np.searchsorted(oracle.E2M1_GRID, q)
-    return (idx | ((v < 0) << 3)).astype(np.uint8)
+    return (idx | (((v < 0) & (idx > 0)) << 3)).astype(np.uint8)
 
 
 def test_e2m1_grid_and_ties():
@@ -198,7 +198,7 @@ def test_e2m1_grid_and_ties():
     mids = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
     assert list(oracle.e2m1_decode(oracle.e2m1_encode(mids))) == [0, 1, 1, 2, 2, 4, 4]
     assert list(oracle.e2m1_encode([6.5, 100.0, -7.0])) == [7, 7, 15]
-    assert list(oracle.e2m1_encode([0.0, -0.0, -0.1, 0.1])) == [0, 0, 8, 0]
+    assert list(oracle.e2m1_encode([0.0, -0.0, -0.1, 0.1, -0.25])) == [0, 0, 0, 0, 0]
 
 
 def test_e2m1_matches_independent_scaled_rounding():
