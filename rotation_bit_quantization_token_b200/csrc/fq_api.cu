@@ -49,10 +49,14 @@ bool mx_rule_from(double d, fq::MxRule* r) {
   return true;
 }
 
-bool use_tc(const fq_handle* h, const void* x, const void* out, const void* scales) {
+// The tensor-core kernel moves x with TMA, P1 / P2 with 16-byte loads and the outputs
+// with bulk copies, so all of them must be 16-byte aligned.
+bool use_tc(const fq_handle* h, const void* x, const void* P1, const void* P2, const void* out,
+            const void* scales) {
   if (h->pref == FQ_KERNEL_GENERAL) return false;
   if (!fq::tc_supported(h->K, h->M, h->N)) return false;
-  return aligned(x, 16) && aligned(out, 16) && (scales == nullptr || aligned(scales, 16));
+  return aligned(x, 16) && aligned(P1, 16) && (P2 == nullptr || aligned(P2, 16)) &&
+         aligned(out, 16) && (scales == nullptr || aligned(scales, 16));
 }
 
 int general_grid(const fq_handle* h) {
@@ -65,7 +69,7 @@ fq_status launch(fq_handle* h, int mode, const void* x, const void* P1, const vo
                  float* x2, cudaStream_t s) {
   const bool fp16_in = h->dtype == FQ_FP16;
   const void* out_probe = (mode == fq::kModeRotate) ? static_cast<const void*>(x2) : out;
-  if (use_tc(h, x, out_probe, mode == fq::kModeMx ? scales : nullptr)) {
+  if (use_tc(h, x, P1, P2, out_probe, mode == fq::kModeMx ? scales : nullptr)) {
     fq::TcParams p{};
     p.x = x; p.P1 = P1; p.P2 = P2; p.K = h->K; p.M = h->M; p.N = h->N; p.mode = mode;
     p.clip_ratio = clip; p.rule = rule; p.out = out; p.quant_scale = qs; p.scales = scales;

@@ -1,7 +1,745 @@
-// Tensor-core kernel placeholder (filled in by the tcgen05 implementation).
+// Tensor-core fused rotate + quantize kernel for sm_100a (tcgen05 / TMEM / TMA).
+//
+// Page: "aclnnFlatQuantV2 complete guide: from two-level matmul to FP4 E2M1
+// quantization fusion" (http://www.zwxr.cn/news/277566): x'' = P1 . (x . P2) per token
+// ("How it works"), then the per-token or per-group quantizer.
+//
+// Layout of the work. Tokens are stacked into 128-row tiles of the [K*M, N] row view of
+// x (128/M tokens per tile, M in {32, 64, 128}). The product is associative, so each
+// tile is computed as
+//     stage A:  Y   = BD(P1) . X        bf16 x bf16 -> fp32 (TMEM), K = 128
+//     stage B:  X'' = Y . P2            Y split as fp16 hi + fp16 lo, fp32 accumulate
+// where BD(P1) is the block-diagonal matrix holding 128/M copies of P1, so one M=128
+// MMA serves every token of the tile. The products of stage A are exact; stage B needs
+// Y, an fp32 value, as a 16-bit operand: each row of Y is scaled by a power of two that
+// puts its largest magnitude in [2^14, 2^15), then split into fp16 hi = rn(y) and
+// lo = rn(y - hi), so hi + lo carries 22 significant bits and the two MMAs of stage B
+// lose nothing beyond float32 rounding. P2 is scaled by one power of two into the same
+// range, converted to fp16 and transposed to K-major once per CTA. The powers of two
+// are undone exactly in the epilogue.
+//
+// Roles (one CTA per SM, persistent over tiles, 320 threads):
+//   warp 0      TMA producer: x tiles (128 rows x N, 128B-swizzled) into a 4-stage ring
+//   warp 1      MMA issuer: stage A (A = BD(P1) in SMEM, B = x tile, MN-major) and
+//               stage B (A = hi/lo Y in TMEM, B = P2^T in SMEM); owns the TMEM
+//   warps 2-5   epilogue group 0 (even local tiles), warps 6-9 group 1 (odd tiles);
+//               each reads its accumulators from TMEM lane = row, writes the split Y back
+//               into TMEM for stage B, then quantizes X'' and stores codes and scales
+//               with bulk async copies from shared memory.
+// Every wait is bounded in time; on expiry the kernel records a code in the status word,
+// drains its copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstdint>
+#include <mutex>
+
 #include "fq_internal.h"
+#include "fq_quant.cuh"
 
 namespace fq {
-bool tc_supported(int64_t, int, int) { return false; }
-cudaError_t launch_tc(const TcParams&, bool, int, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+constexpr int kStages = 4;
+constexpr int kThreads = 320;
+constexpr uint64_t kTimeoutNs = 4000000000ull;  // 4 s: far beyond any legitimate wait
+
+// status bits (device status word)
+enum : uint32_t {
+  kStProducerEmpty = 1u << 0, kStMmaXFull = 1u << 1, kStMmaTmemEmpty = 1u << 2,
+  kStMmaYsFull = 1u << 3, kStEpiAFull = 1u << 4, kStEpiBFull = 1u << 5,
+  kStMmaDone = 1u << 6, kStDrain = 1u << 7
+};
+
+template <int N>
+struct Geo {
+  static_assert(N % 16 == 0 && N >= 64 && N <= 128, "tensor-core kernel covers N in [64,128], N % 16 == 0");
+  static constexpr int kAtoms = (N + 63) / 64;              // 64-element swizzle atoms along N
+  static constexpr int kXStage = kAtoms * 128 * 128;        // bytes per x stage
+  static constexpr int kP1Bytes = 2 * 128 * 128;            // BD(P1): 128 x 128, two K atoms
+  static constexpr int kP2Bytes = kAtoms * N * 128;         // P2^T: N rows, kAtoms K atoms
+  static constexpr int kCodeBytes = 128 * N / 2;
+  static constexpr int kScaleBytes = 4 * N;                 // 128 rows x N/32 groups
+  static constexpr int kOutStride = (kCodeBytes + kScaleBytes + 1023) & ~1023;
+  static constexpr int kOffP1 = 0;
+  static constexpr int kOffP2 = kOffP1 + kP1Bytes;
+  static constexpr int kOffX = kOffP2 + kP2Bytes;
+  static constexpr int kOffOut = kOffX + kStages * kXStage;
+  static constexpr int kOffBar = kOffOut + 2 * kOutStride;
+  static constexpr int kSmem = kOffBar + 512 + 1024;        // + alignment slack
+  static constexpr uint32_t kTmemCols = (4 * N <= 256) ? 256u : 512u;
+};
+
+struct Bars {
+  uint64_t x_full[kStages];
+  uint64_t x_empty[kStages];
+  uint64_t da_full[2];
+  uint64_t ys_full[2];
+  uint64_t db_full[2];
+  uint64_t tm_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort;
+  int group_exit[2];
+  float red[2][4];
+  float wmax[kThreads / 32];
+};
+
+// ------------------------------------------------------------------------------------
+// PTX wrappers
+// ------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(b), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void named_bar(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor (tcgen05): start, leading / stride byte offsets,
+// version 1, 128-byte swizzle.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr >> 4) & 0x3FFFu);
+  d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
+  d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
+  d |= uint64_t(1) << 46;
+  d |= uint64_t(2) << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16, fp32 accumulate, M = 128.
+__host__ __device__ constexpr uint32_t idesc_f16(bool a_bf16, bool b_bf16, bool b_mn_major, int n) {
+  return (1u << 4) | (uint32_t(a_bf16) << 7) | (uint32_t(b_bf16) << 10) |
+         (uint32_t(b_mn_major) << 16) | (uint32_t(n >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+}
+
+// 2^e as float32 for e in [-149, 127] (clamped).
+__device__ __forceinline__ float exp2i(int e) {
+  e = e < -149 ? -149 : (e > 127 ? 127 : e);
+  return e >= -126 ? __int_as_float((e + 127) << 23) : __int_as_float(1 << (e + 149));
+}
+
+// Exponent s with m * 2^s in [2^14, 2^15) for a positive normal m (clamped to the
+// normal range of the factor); 0 for zero or non-finite m.
+__device__ __forceinline__ int prescale_exp(float m) {
+  const uint32_t E = (__float_as_uint(m) >> 23) & 0xFFu;
+  if (m == 0.0f || E == 0xFFu) return 0;
+  int s = 141 - int(E == 0 ? 1 : E);
+  return s < -126 ? -126 : (s > 127 ? 127 : s);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Bounded wait on an mbarrier phase. On expiry sets the abort flag and a status bit.
+__device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, Bars* bars, uint32_t* status,
+                                          uint32_t code) {
+  const uint32_t b = smem_u32(bar);
+  if (mbar_try_wait(b, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(b, parity)) return true;
+    if ((it & 63u) == 0u) {
+      if (*reinterpret_cast<volatile int*>(&bars->abort)) return false;
+      if (globaltimer() - t0 > kTimeoutNs) {
+        *reinterpret_cast<volatile int*>(&bars->abort) = 1;
+        atomicOr(status, code);
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait used by whole warps: uniform result across the warp.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Bars* bars, uint32_t* status,
+                                          uint32_t code) {
+  const bool ok = wait_bounded(bar, parity, bars, status, code);
+  return __all_sync(0xffffffffu, ok);
+}
+
+template <bool kF16>
+__device__ __forceinline__ float ld16f(const void* base, int i) {
+  const uint16_t u = static_cast<const uint16_t*>(base)[i];
+  if constexpr (kF16) return __half2float(__ushort_as_half(u));
+  else return __bfloat162float(__ushort_as_bfloat16(u));
+}
+
+template <bool kF16>
+__device__ __forceinline__ void unpack8(const uint4& q, float* f) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if constexpr (kF16) {
+      const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+      f[2 * i] = t.x;
+      f[2 * i + 1] = t.y;
+    } else {
+      const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+      f[2 * i] = t.x;
+      f[2 * i + 1] = t.y;
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+
+// ------------------------------------------------------------------------------------
+// the kernel
+// ------------------------------------------------------------------------------------
+template <int N, bool kF16, int kMode>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
+  using G = Geo<N>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars* bars = reinterpret_cast<Bars*>(smem + G::kOffBar);
+  const uint32_t sbase = smem_u32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int M = p.M;
+  const int64_t rows_total = p.K * int64_t(M);
+  const int num_tiles = int((rows_total + 127) / 128);
+
+  // ---- prologue: P2 scale, BD(P1) and P2^T operands, barriers, TMEM ----
+  float lmax = 0.0f;
+  if (p.P2 != nullptr) {
+    for (int i = tid; i < N * N; i += kThreads) lmax = fmaxf(lmax, fabsf(ld16f<kF16>(p.P2, i)));
+  } else {
+    lmax = 1.0f;
+  }
+  lmax = warp_max(lmax);
+  if (lane == 0) bars->wmax[warp] = lmax;
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->x_full[s], 1);
+      mbar_init(&bars->x_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->da_full[b], 1);
+      mbar_init(&bars->ys_full[b], 4);
+      mbar_init(&bars->db_full[b], 1);
+      mbar_init(&bars->tm_empty[b], 4);
+    }
+    mbar_init(&bars->mma_done, 1);
+    bars->abort = 0;
+    bars->group_exit[0] = bars->group_exit[1] = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  float p2max = 0.0f;
+#pragma unroll
+  for (int w = 0; w < kThreads / 32; ++w) p2max = fmaxf(p2max, bars->wmax[w]);
+  const int t_exp = prescale_exp(p2max);
+  const float p2scale = exp2i(t_exp);
+
+  // BD(P1): 128 x 128, K-major, 128B swizzle; element (r, k) = P1[r % M][k % M] on the
+  // diagonal blocks (r / M == k / M), else 0.
+  for (int c = tid; c < 128 * 16; c += kThreads) {
+    const int r = c >> 4, kc = c & 15, k = kc * 8;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (r / M == k / M)
+      v = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.P1) + (r % M) * M + (k % M));
+    const uint32_t off = G::kOffP1 + (kc >> 3) * 16384 + r * 128 + ((((kc & 7) ^ (r & 7))) << 4);
+    *reinterpret_cast<uint4*>(smem + off) = v;
+  }
+  // P2^T scaled by 2^t as fp16: N rows (n), K = N (j), K-major, 128B swizzle.
+  constexpr int NB = N / 8;
+  for (int blk = tid; blk < NB * NB; blk += kThreads) {
+    const int jb = blk / NB, nb = blk % NB;
+    float v[8][8];
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      const int j = jb * 8 + jj;
+      if (p.P2 != nullptr) {
+        const uint4 q = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.P2) + j * N + nb * 8);
+        unpack8<kF16>(q, v[jj]);
+      } else {
+#pragma unroll
+        for (int nn = 0; nn < 8; ++nn) v[jj][nn] = (j == nb * 8 + nn) ? 1.0f : 0.0f;
+      }
+    }
+#pragma unroll
+    for (int nn = 0; nn < 8; ++nn) {
+      const int n = nb * 8 + nn;
+      uint32_t w[4];
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj)
+        w[jj] = h2_bits(__floats2half2_rn(v[2 * jj][nn] * p2scale, v[2 * jj + 1][nn] * p2scale));
+      const uint32_t off = G::kOffP2 + (jb >> 3) * (N * 128) + n * 128 + ((((jb & 7) ^ (n & 7))) << 4);
+      *reinterpret_cast<uint4*>(smem + off) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+  fence_proxy_async();
+  if (warp == 1) tmem_alloc(&bars->tmem_base, G::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int i = 0;
+      int last_i[kStages];
+#pragma unroll
+      for (int s = 0; s < kStages; ++s) last_i[s] = -1;
+      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
+        const int s = i % kStages;
+        if (!wait_bounded(&bars->x_empty[s], ((i / kStages) & 1) ^ 1, bars, p.status, kStProducerEmpty)) break;
+        mbar_arrive_expect_tx(&bars->x_full[s], G::kXStage);
+#pragma unroll
+        for (int a = 0; a < G::kAtoms; ++a)
+          tma_load_2d(sbase + G::kOffX + s * G::kXStage + a * 16384, &tmap, a * 64, tile * 128,
+                      &bars->x_full[s]);
+        last_i[s] = i;
+      }
+      // drain: every issued load has landed before the CTA may exit
+      for (int s = 0; s < kStages; ++s) {
+        if (last_i[s] < 0) continue;
+        const uint32_t b = smem_u32(&bars->x_full[s]);
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(b, (last_i[s] / kStages) & 1)) {
+          if (globaltimer() - t0 > kTimeoutNs) { atomicOr(p.status, kStDrain); break; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const int n_local = (blockIdx.x < num_tiles) ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+      constexpr uint32_t kIdA = idesc_f16(!kF16, !kF16, true, N);
+      constexpr uint32_t kIdB = idesc_f16(false, false, false, N);
+      auto issue_a = [&](int i) -> bool {
+        const int s = i % kStages, b = i & 1, j = i >> 1;
+        if (!wait_bounded(&bars->x_full[s], (i / kStages) & 1, bars, p.status, kStMmaXFull)) return false;
+        if (!wait_bounded(&bars->tm_empty[b], (j & 1) ^ 1, bars, p.status, kStMmaTmemEmpty)) return false;
+        tc_fence_after();
+        const uint32_t d = tmem + uint32_t(b * 2 * N);
+        const uint32_t xs = sbase + G::kOffX + s * G::kXStage;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t a = sdesc(sbase + G::kOffP1 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t bx = sdesc(xs + kk * 2048, 16384, 1024);
+          mma_ss(d, a, bx, kIdA, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars->x_empty[s]);
+        mma_commit(&bars->da_full[b]);
+        return true;
+      };
+      auto issue_b = [&](int i) -> bool {
+        const int b = i & 1, j = i >> 1;
+        if (!wait_bounded(&bars->ys_full[b], j & 1, bars, p.status, kStMmaYsFull)) return false;
+        tc_fence_after();
+        const uint32_t d = tmem + uint32_t(b * 2 * N + N);
+        const uint32_t a0 = tmem + uint32_t(b * 2 * N);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int kk = 0; kk < N / 16; ++kk) {
+            const uint64_t bp = sdesc(sbase + G::kOffP2 + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024);
+            mma_ts(d, a0 + uint32_t(h * (N / 2) + kk * 8), bp, kIdB, (h | kk) != 0 ? 1u : 0u);
+          }
+        }
+        mma_commit(&bars->db_full[b]);
+        return true;
+      };
+      bool ok = true;
+      for (int i = 0; ok && i < n_local; ++i) {
+        ok = issue_a(i);
+        if (ok && i >= 1) ok = issue_b(i - 1);
+      }
+      if (ok && n_local >= 1) issue_b(n_local - 1);
+      // every MMA issued above has completed before TMEM is released
+      mma_commit(&bars->mma_done);
+      const uint32_t b = smem_u32(&bars->mma_done);
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(b, 0)) {
+        if (globaltimer() - t0 > kTimeoutNs) { atomicOr(p.status, kStMmaDone); break; }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue groups ----------------
+    const int g = (warp - 2) >> 2;        // group
+    const int q = warp & 3;               // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;        // tile row owned by this thread
+    const uint32_t t_lane = tmem + (uint32_t(q * 32) << 16);
+    const uint32_t colA = uint32_t(g * 2 * N), colB = colA + N;
+    uint8_t* s_out = smem + G::kOffOut + g * G::kOutStride;
+    const uint32_t s_out_u32 = sbase + G::kOffOut + g * G::kOutStride;
+    const bool leader = (warp == 2 + 4 * g) && lane == 0;
+    const int bar_id = 1 + g;
+    const int tok_in_tile = row / M;
+    const int m_row = row % M;
+
+    int i = g;
+    for (int tile = blockIdx.x + g * gridDim.x; tile < num_tiles; tile += 2 * gridDim.x, i += 2) {
+      const int j = i >> 1;
+      const int64_t grow = int64_t(tile) * 128 + row;
+      const int64_t rows_left = rows_total - int64_t(tile) * 128;
+      const int valid_rows = rows_left < 128 ? int(rows_left) : 128;
+
+      // ---- phase 1: Y -> per-row power-of-two scale -> fp16 hi / lo back into TMEM ----
+      int s_exp = 0;
+      const bool ok1 = warp_wait(&bars->da_full[g], j & 1, bars, p.status, kStEpiAFull);
+      if (ok1) {
+        tc_fence_after();
+        float y[N];
+#pragma unroll
+        for (int c = 0; c < N / 16; ++c) tmem_ld16(t_lane + colA + c * 16, y + c * 16);
+        tmem_wait_ld();
+        float rmax = 0.0f;
+#pragma unroll
+        for (int e = 0; e < N; ++e) rmax = fmaxf(rmax, fabsf(y[e]));
+        s_exp = prescale_exp(rmax);
+        const float sc = exp2i(s_exp);
+#pragma unroll
+        for (int c = 0; c < N / 16; ++c) {
+          uint32_t hw[8], lw[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float a = y[c * 16 + 2 * e] * sc, b = y[c * 16 + 2 * e + 1] * sc;
+            const __half2 h = __floats2half2_rn(a, b);
+            const float2 hf = __half22float2(h);
+            hw[e] = h2_bits(h);
+            lw[e] = h2_bits(__floats2half2_rn(a - hf.x, b - hf.y));
+          }
+          tmem_st8(t_lane + colA + c * 8, hw);
+          tmem_st8(t_lane + colA + N / 2 + c * 8, lw);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->ys_full[g]);
+
+      // ---- phase 2: X'' = D * 2^crow, quantize ----
+      float d[N];
+      const bool ok2 = warp_wait(&bars->db_full[g], j & 1, bars, p.status, kStEpiBFull);
+      if (ok2) {
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < N / 16; ++c) tmem_ld16(t_lane + colB + c * 16, d + c * 16);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < N; ++e) d[e] = 0.0f;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->tm_empty[g]);
+
+      const int crow = -(s_exp + t_exp);
+      const float fcrow = exp2i(crow);
+      const bool row_valid = grow < rows_total;
+
+      if constexpr (kMode == kModeRotate) {
+        if (row_valid) {
+          float4* dst = reinterpret_cast<float4*>(p.x2 + grow * N);
+#pragma unroll
+          for (int e = 0; e < N; e += 4)
+            dst[e / 4] = make_float4(d[e] * fcrow, d[e + 1] * fcrow, d[e + 2] * fcrow, d[e + 3] * fcrow);
+        }
+        if (leader) bars->group_exit[g] = *reinterpret_cast<volatile int*>(&bars->abort);
+        named_bar(bar_id, 128);
+        if (bars->group_exit[g]) break;
+        continue;
+      } else {
+        uint32_t words[N / 8];
+        if constexpr (kMode == kModePerToken) {
+          float rmax = 0.0f;
+#pragma unroll
+          for (int e = 0; e < N; ++e) rmax = fmaxf(rmax, fabsf(d[e]));
+          const float wm = warp_max(rmax * fcrow);
+          if (lane == 0) bars->red[g][q] = wm;
+          if (leader) bulk_wait_read0();
+          named_bar(bar_id, 128);
+          float amax = 0.0f;
+          const int q0 = (tok_in_tile * M) >> 5, nq = (M + 31) >> 5;
+          for (int qq = 0; qq < nq; ++qq) amax = fmaxf(amax, bars->red[g][q0 + qq]);
+          const float qs = per_token_scale(amax, p.clip_ratio);
+          const float inv = qs > 0.0f ? __frcp_rn(qs) : 0.0f;
+          const float F = inv * fcrow;
+          if (row_valid && m_row == 0) p.quant_scale[grow / M] = qs;
+#pragma unroll
+          for (int w = 0; w < N / 8; ++w) {
+            uint32_t acc = 0u;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float v = fminf(fmaxf(d[w * 8 + e] * F, -8.0f), 7.0f);
+              acc |= (uint32_t(__float2int_rn(v)) & 0xFu) << (4 * e);
+            }
+            words[w] = acc;
+          }
+        } else {
+          // per-group E2M1: segment maxima over 16 columns, groups of 32 in the flattened
+          // token; when N % 32 == 16 a row pair (2r, 2r+1) shares one group across the
+          // row end, combined through a lane shuffle (the pair sits in adjacent lanes).
+          constexpr int NS = N / 16;
+          float smax[NS];
+#pragma unroll
+          for (int sgi = 0; sgi < NS; ++sgi) {
+            float m = 0.0f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) m = fmaxf(m, fabsf(d[sgi * 16 + e]));
+            smax[sgi] = m;
+          }
+          float Fseg[NS];
+          uint8_t* s_scale = s_out + G::kCodeBytes;
+          if (leader) bulk_wait_read0();
+          named_bar(bar_id, 128);
+          if constexpr ((N % 32) == 0) {
+#pragma unroll
+            for (int gi = 0; gi < NS / 2; ++gi) {
+              const float amax = fmaxf(smax[2 * gi], smax[2 * gi + 1]) * fcrow;
+              const MxScale ms = mx_scale(amax, p.rule);
+              const float F = exp2i(127 - int(ms.byte) + crow);
+              Fseg[2 * gi] = F;
+              Fseg[2 * gi + 1] = F;
+              s_scale[row * (N / 32) + gi] = uint8_t(ms.byte);
+            }
+          } else {
+            constexpr int GF = (N - 16) / 32;  // full groups per row
+            const bool odd = (row & 1) != 0;
+            // the straddling half-group: last 16 columns of an even row, first 16 of an odd row
+            const float part = (odd ? smax[0] : smax[NS - 1]) * fcrow;
+            const float other = __shfl_xor_sync(0xffffffffu, part, 1);
+            const MxScale mst = mx_scale(fmaxf(part, other), p.rule);
+            const float Fst = exp2i(127 - int(mst.byte) + crow);
+            const int pair_base = (row >> 1) * (N / 16);
+            float Ff[GF];
+#pragma unroll
+            for (int gi = 0; gi < GF; ++gi) {
+              const float a = odd ? fmaxf(smax[2 * gi + 1], smax[2 * gi + 2]) : fmaxf(smax[2 * gi], smax[2 * gi + 1]);
+              const MxScale ms = mx_scale(a * fcrow, p.rule);
+              Ff[gi] = exp2i(127 - int(ms.byte) + crow);
+              s_scale[pair_base + (odd ? GF + 1 : 0) + gi] = uint8_t(ms.byte);
+            }
+            if (!odd) s_scale[pair_base + GF] = uint8_t(mst.byte);
+#pragma unroll
+            for (int sgi = 0; sgi < NS; ++sgi) {
+              const float fe = (sgi == NS - 1) ? Fst : Ff[sgi >> 1];
+              const float fo = (sgi == 0) ? Fst : Ff[(sgi - 1) >> 1];
+              Fseg[sgi] = odd ? fo : fe;
+            }
+          }
+#pragma unroll
+          for (int w = 0; w < N / 8; ++w) {
+            const float F = Fseg[w >> 1];
+            uint32_t acc = 0u;
+#pragma unroll
+            for (int e = 0; e < 8; e += 2)
+              acc |= e2m1x2_raw(d[w * 8 + e] * F, d[w * 8 + e + 1] * F) << (4 * e);
+            words[w] = e2m1_canonical_zero(acc);
+          }
+        }
+        // codes of this row: N/2 bytes at row * N/2 in the staging buffer
+        if constexpr ((N % 32) == 0) {
+          uint4* dst = reinterpret_cast<uint4*>(s_out + row * (N / 2));
+#pragma unroll
+          for (int w = 0; w < N / 8; w += 4) dst[w / 4] = make_uint4(words[w], words[w + 1], words[w + 2], words[w + 3]);
+        } else {
+          uint2* dst = reinterpret_cast<uint2*>(s_out + row * (N / 2));
+#pragma unroll
+          for (int w = 0; w < N / 8; w += 2) dst[w / 2] = make_uint2(words[w], words[w + 1]);
+        }
+        fence_proxy_async();
+        if (leader) bars->group_exit[g] = *reinterpret_cast<volatile int*>(&bars->abort);
+        named_bar(bar_id, 128);
+        if (leader) {
+          const int64_t row0 = int64_t(tile) * 128;
+          bulk_store(p.out + row0 * (N / 2), s_out_u32, uint32_t(valid_rows * (N / 2)));
+          if constexpr (kMode == kModeMx)
+            bulk_store(p.scales + (row0 * N) / 32, s_out_u32 + G::kCodeBytes, uint32_t((valid_rows * N) / 32));
+          bulk_commit();
+        }
+        if (bars->group_exit[g]) break;
+      }
+    }
+    if (leader) bulk_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, G::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// host side
+// ------------------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+template <int N, bool kF16, int kMode>
+cudaError_t launch_n(const TcParams& p, int num_sms, cudaStream_t stream) {
+  using G = Geo<N>;
+  auto enc = get_encode();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {cuuint64_t(N), cuuint64_t(p.K * p.M)};
+  const cuuint64_t strides[1] = {cuuint64_t(N) * 2};
+  const cuuint32_t box[2] = {64u, 128u};
+  const cuuint32_t estr[2] = {1u, 1u};
+  const CUresult r = enc(&map, kF16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                         const_cast<void*>(p.x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  auto kern = tc_kernel<N, kF16, kMode>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::kSmem);
+  if (e != cudaSuccess) return e;
+  const int64_t tiles = (p.K * p.M + 127) / 128;
+  const int grid = int(tiles < num_sms ? tiles : num_sms);
+  kern<<<grid, kThreads, G::kSmem, stream>>>(map, p);
+  return cudaGetLastError();
+}
+
+template <int N>
+cudaError_t launch_mode(const TcParams& p, bool f16, int sms, cudaStream_t s) {
+  if (p.mode == kModePerToken)
+    return f16 ? launch_n<N, true, kModePerToken>(p, sms, s) : launch_n<N, false, kModePerToken>(p, sms, s);
+  if (p.mode == kModeMx)
+    return f16 ? launch_n<N, true, kModeMx>(p, sms, s) : launch_n<N, false, kModeMx>(p, sms, s);
+  return f16 ? launch_n<N, true, kModeRotate>(p, sms, s) : launch_n<N, false, kModeRotate>(p, sms, s);
+}
+
+}  // namespace
+
+bool tc_supported(int64_t K, int M, int N) {
+  (void)K;
+  return (M == 32 || M == 64 || M == 128) && (N % 16 == 0) && N >= 64 && N <= 128;
+}
+
+cudaError_t launch_tc(const TcParams& p, bool fp16_in, int num_sms, cudaStream_t stream) {
+  switch (p.N) {
+    case 64: return launch_mode<64>(p, fp16_in, num_sms, stream);
+    case 80: return launch_mode<80>(p, fp16_in, num_sms, stream);
+    case 96: return launch_mode<96>(p, fp16_in, num_sms, stream);
+    case 112: return launch_mode<112>(p, fp16_in, num_sms, stream);
+    case 128: return launch_mode<128>(p, fp16_in, num_sms, stream);
+    default: return cudaErrorNotSupported;
+  }
+}
+
 }  // namespace fq
