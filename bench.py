@@ -44,6 +44,9 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default=BENCH_WORKLOAD, choices=sorted(WORKLOADS))
     p.add_argument("--kernel", default="auto", choices=["auto", "general", "tcgen05"])
+    p.add_argument("--tokens", type=int, default=0,
+                   help="override the token count (a smaller case of the same workload, "
+                        "for profiling); 0 keeps the workload's own K")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
@@ -244,6 +247,8 @@ def run_ours(args, rank, world, local):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=dev)
     w = WORKLOADS[args.workload]
+    if args.tokens:
+        w = w.with_tokens(args.tokens)
     # cpu baseline first (rank 0 at N = 1 only), while nothing runs on the GPU
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
