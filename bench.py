@@ -195,6 +195,11 @@ def bounded_oracle_sample(w, seed, target_s=12.0, min_tokens=16, max_tokens=4096
     while dt < target_s / 8 and n < xf.shape[0]:
         n = min(xf.shape[0], n * 4)
         dt = run(n)
+    # final sample sized to about target_s of work (bounded by the tokens drawn)
+    n_final = int(min(xf.shape[0], max(n, n * target_s / max(dt, 1e-9))))
+    if n_final > n:
+        n = n_final
+        dt = run(n)
     threads = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
     return n / dt, n, dt, threads
 
