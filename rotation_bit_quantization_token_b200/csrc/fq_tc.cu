@@ -14,18 +14,23 @@
 // Y, an fp32 value, as a 16-bit operand: each row of Y is scaled by a power of two that
 // puts its largest magnitude in [2^14, 2^15), then split into fp16 hi = rn(y) and
 // lo = rn(y - hi), so hi + lo carries 22 significant bits and the two MMAs of stage B
-// lose nothing beyond float32 rounding. P2 is scaled by one power of two into the same
+// lose nothing beyond float32 rounding. In TMEM each 16-column block of a row of Y is
+// replaced by the 8 words of hi followed by the 8 words of lo of the same 16 elements. P2 is scaled by one power of two into the same
 // range, converted to fp16 and transposed to K-major once per CTA. The powers of two
 // are undone exactly in the epilogue.
 //
-// Roles (one CTA per SM, persistent over tiles, 320 threads):
-//   warp 0      TMA producer: x tiles (128 rows x N, 128B-swizzled) into a 4-stage ring
-//   warp 1      MMA issuer: stage A (A = BD(P1) in SMEM, B = x tile, MN-major) and
+// Roles (one CTA per SM, persistent over tiles, 384 threads = 3 warpgroups):
+//   warps 0-3   splitter: reads Y from TMEM (lane = row), scales each row by a power of
+//               two, writes fp16 hi / lo back into the same TMEM columns for stage B
+//   warps 4-7   quantizer: reads X'' from TMEM, forms per-token or per-group scales and
+//               codes, stages them in shared memory and stores them with bulk copies
+//               (double-buffered staging)
+//   warp 8      TMA producer: x tiles (128 rows x N, 128B-swizzled) into a 4-stage ring
+//   warp 9      MMA issuer: stage A (A = BD(P1) in SMEM, B = x tile, MN-major) and
 //               stage B (A = hi/lo Y in TMEM, B = P2^T in SMEM); owns the TMEM
-//   warps 2-5   epilogue group 0 (even local tiles), warps 6-9 group 1 (odd tiles);
-//               each reads its accumulators from TMEM lane = row, writes the split Y back
-//               into TMEM for stage B, then quantizes X'' and stores codes and scales
-//               with bulk async copies from shared memory.
+//   warps 10-11 idle after the prologue
+// Two TMEM buffers (D_A for Y, D_B for X'') let stage A of tile i+2 run while the
+// quantizer still reads tile i.
 // Every wait is bounded in time; on expiry the kernel records a code in the status word,
 // drains its copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -43,7 +48,13 @@ namespace fq {
 namespace {
 
 constexpr int kStages = 4;
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;  // three warpgroups
+// Register split (setmaxnreg): launched at kLaunchRegs per thread; the producer / MMA
+// warpgroup drops to kLowRegs and the two epilogue warpgroups rise to kHighRegs, using
+// exactly the registers the block was launched with:
+// 2 * 128 * kHighRegs + 128 * kLowRegs == kThreads * kLaunchRegs.
+constexpr int kLaunchRegs = 168, kLowRegs = 56, kHighRegs = 224;
+static_assert(2 * 128 * kHighRegs + 128 * kLowRegs == kThreads * kLaunchRegs, "register split");
 constexpr uint64_t kTimeoutNs = 4000000000ull;  // 4 s: far beyond any legitimate wait
 
 // status bits (device status word)
@@ -68,7 +79,7 @@ struct Geo {
   static constexpr int kOffX = kOffP2 + kP2Bytes;
   static constexpr int kOffOut = kOffX + kStages * kXStage;
   static constexpr int kOffBar = kOffOut + 2 * kOutStride;
-  static constexpr int kSmem = kOffBar + 512 + 1024;        // + alignment slack
+  static constexpr int kSmem = kOffBar + 1024 + 1024;       // barriers + alignment slack
   static constexpr uint32_t kTmemCols = (4 * N <= 256) ? 256u : 512u;
 };
 
@@ -79,12 +90,14 @@ struct Bars {
   uint64_t ys_full[2];
   uint64_t db_full[2];
   uint64_t tm_empty[2];
+  uint64_t srow_full[4];  // row exponents of tile i published in srow[i % 4]
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
-  int group_exit[2];
+  int group_exit[2];  // quantizer exit decision, one slot per tile parity
   float red[2][4];
   float wmax[kThreads / 32];
+  int8_t srow[4][128];  // per-row power-of-two exponent of Y, ring of four tiles
 };
 
 // ------------------------------------------------------------------------------------
@@ -133,9 +146,6 @@ __device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc, uint32_t b
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read0() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -192,10 +202,11 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
   asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
@@ -240,8 +251,65 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
+// max(|a|, |b|, |c|) in one instruction
+__device__ __forceinline__ float max3abs(float a, float b, float c) {
+  float r;
+  asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// largest magnitude of n values (n a multiple of 16) as a shallow tree
+template <int n>
+__device__ __forceinline__ float absmax(const float* v) {
+  float acc[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) acc[k] = 0.0f;
+#pragma unroll
+  for (int e = 0; e < n; e += 2) acc[(e >> 1) & 7] = max3abs(acc[(e >> 1) & 7], v[e], v[e + 1]);
+  const float a = max3abs(acc[0], acc[1], acc[2]);
+  const float b = max3abs(acc[3], acc[4], acc[5]);
+  return max3abs(a, b, fmaxf(acc[6], acc[7]));
+}
+__device__ __forceinline__ float absmax16(const float* v) {
+  const float a = max3abs(v[0], v[1], v[2]), b = max3abs(v[3], v[4], v[5]);
+  const float c = max3abs(v[6], v[7], v[8]), d = max3abs(v[9], v[10], v[11]);
+  const float e = max3abs(v[12], v[13], v[14]);
+  return fmaxf(max3abs(a, b, c), max3abs(d, e, v[15]));
+}
+// insert the low 4 bits of src into acc at bit position pos
+__device__ __forceinline__ uint32_t bfi4(uint32_t src, uint32_t acc, int pos) {
+  uint32_t r;
+  asm("bfi.b32 %0, %1, %2, %3, 4;" : "=r"(r) : "r"(src), "r"(acc), "r"(pos));
+  return r;
+}
+// eight E2M1 codes (round to nearest even, saturate) in one word: element 0 in bits 0-3
+__device__ __forceinline__ uint32_t e2m1x8(float2 a, float2 b, float2 c, float2 d) {
+  uint32_t r;
+  // cvt puts its first source in the upper nibble of each byte
+  asm("{\n\t.reg .b8 t0, t1, t2, t3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t3, %8, %7;\n\t"
+      "mov.b32 %0, {t0, t1, t2, t3};\n\t}"
+      : "=r"(r)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y), "f"(d.x), "f"(d.y));
+  return r;
+}
+template <int n>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(n) : "memory");
+}
+
+template <int n>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(n));
+}
+template <int n>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(n));
+}
 // Bounded wait on an mbarrier phase. On expiry sets the abort flag and a status bit.
-__device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, Bars* bars, uint32_t* status,
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, Bars* bars, uint32_t* status,
                                           uint32_t code) {
   const uint32_t b = smem_u32(bar);
   if (mbar_try_wait(b, parity)) return true;
@@ -328,6 +396,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       mbar_init(&bars->db_full[b], 1);
       mbar_init(&bars->tm_empty[b], 4);
     }
+    for (int r = 0; r < 4; ++r) mbar_init(&bars->srow_full[r], 4);
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
     bars->group_exit[0] = bars->group_exit[1] = 0;
@@ -378,14 +447,15 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     }
   }
   fence_proxy_async();
-  if (warp == 1) tmem_alloc(&bars->tmem_base, G::kTmemCols);
+  if (warp == 9) tmem_alloc(&bars->tmem_base, G::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == 0) {
+  if (warp == 8) {
     // ---------------- TMA producer ----------------
+    setmaxnreg_dec<kLowRegs>();
     if (lane == 0) {
       int i = 0;
       int last_i[kStages];
@@ -411,8 +481,12 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 9) {
     // ---------------- MMA issuer ----------------
+    setmaxnreg_dec<kLowRegs>();
+    // Order A(i), A(i+1), B(i), B(i+1): stage A of the next pair is issued while stage B
+    // of this pair runs. A(i) may overwrite D_A[b] once B(i-2) has read its hi / lo Y;
+    // B(i) may overwrite D_B[b] once the quantizer has read the X'' of tile i-2.
     if (lane == 0) {
       const int n_local = (blockIdx.x < num_tiles) ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
       constexpr uint32_t kIdA = idesc_f16(!kF16, !kF16, true, N);
@@ -420,7 +494,8 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       auto issue_a = [&](int i) -> bool {
         const int s = i % kStages, b = i & 1, j = i >> 1;
         if (!wait_bounded(&bars->x_full[s], (i / kStages) & 1, bars, p.status, kStMmaXFull)) return false;
-        if (!wait_bounded(&bars->tm_empty[b], (j & 1) ^ 1, bars, p.status, kStMmaTmemEmpty)) return false;
+        if (j >= 1 && !wait_bounded(&bars->db_full[b], (j - 1) & 1, bars, p.status, kStMmaTmemEmpty))
+          return false;
         tc_fence_after();
         const uint32_t d = tmem + uint32_t(b * 2 * N);
         const uint32_t xs = sbase + G::kOffX + s * G::kXStage;
@@ -437,6 +512,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       auto issue_b = [&](int i) -> bool {
         const int b = i & 1, j = i >> 1;
         if (!wait_bounded(&bars->ys_full[b], j & 1, bars, p.status, kStMmaYsFull)) return false;
+        if (!wait_bounded(&bars->tm_empty[b], (j & 1) ^ 1, bars, p.status, kStMmaTmemEmpty)) return false;
         tc_fence_after();
         const uint32_t d = tmem + uint32_t(b * 2 * N + N);
         const uint32_t a0 = tmem + uint32_t(b * 2 * N);
@@ -445,18 +521,19 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
 #pragma unroll
           for (int kk = 0; kk < N / 16; ++kk) {
             const uint64_t bp = sdesc(sbase + G::kOffP2 + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024);
-            mma_ts(d, a0 + uint32_t(h * (N / 2) + kk * 8), bp, kIdB, (h | kk) != 0 ? 1u : 0u);
+            mma_ts(d, a0 + uint32_t(kk * 16 + h * 8), bp, kIdB, (h | kk) != 0 ? 1u : 0u);
           }
         }
         mma_commit(&bars->db_full[b]);
         return true;
       };
       bool ok = true;
-      for (int i = 0; ok && i < n_local; ++i) {
+      for (int i = 0; ok && i < n_local; i += 2) {
         ok = issue_a(i);
-        if (ok && i >= 1) ok = issue_b(i - 1);
+        if (ok && i + 1 < n_local) ok = issue_a(i + 1);
+        if (ok) ok = issue_b(i);
+        if (ok && i + 1 < n_local) ok = issue_b(i + 1);
       }
-      if (ok && n_local >= 1) issue_b(n_local - 1);
       // every MMA issued above has completed before TMEM is released
       mma_commit(&bars->mma_done);
       const uint32_t b = smem_u32(&bars->mma_done);
@@ -466,68 +543,88 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       }
     }
     __syncwarp();
-  } else {
-    // ---------------- epilogue groups ----------------
-    const int g = (warp - 2) >> 2;        // group
-    const int q = warp & 3;               // TMEM lane quarter this warp may access
-    const int row = q * 32 + lane;        // tile row owned by this thread
+  } else if (warp >= 10) {
+    setmaxnreg_dec<kLowRegs>();  // idle warps of the producer / MMA warpgroup
+  } else if (warp < 4) {
+    // ---------------- splitter: Y -> per-row power-of-two scale -> fp16 hi / lo ----------------
+    setmaxnreg_inc<kHighRegs>();
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
     const uint32_t t_lane = tmem + (uint32_t(q * 32) << 16);
-    const uint32_t colA = uint32_t(g * 2 * N), colB = colA + N;
-    uint8_t* s_out = smem + G::kOffOut + g * G::kOutStride;
-    const uint32_t s_out_u32 = sbase + G::kOffOut + g * G::kOutStride;
-    const bool leader = (warp == 2 + 4 * g) && lane == 0;
-    const int bar_id = 1 + g;
-    const int tok_in_tile = row / M;
-    const int m_row = row % M;
-
-    int i = g;
-    for (int tile = blockIdx.x + g * gridDim.x; tile < num_tiles; tile += 2 * gridDim.x, i += 2) {
-      const int j = i >> 1;
-      const int64_t grow = int64_t(tile) * 128 + row;
-      const int64_t rows_left = rows_total - int64_t(tile) * 128;
-      const int valid_rows = rows_left < 128 ? int(rows_left) : 128;
-
-      // ---- phase 1: Y -> per-row power-of-two scale -> fp16 hi / lo back into TMEM ----
+    int i = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
+      const int b = i & 1, j = i >> 1;
+      const uint32_t colA = uint32_t(b * 2 * N);
       int s_exp = 0;
-      const bool ok1 = warp_wait(&bars->da_full[g], j & 1, bars, p.status, kStEpiAFull);
-      if (ok1) {
+      const bool ok = warp_wait(&bars->da_full[b], j & 1, bars, p.status, kStEpiAFull);
+      if (ok) {
         tc_fence_after();
+        // one TMEM round trip: the whole row, then the row maximum as a shallow tree
         float y[N];
 #pragma unroll
         for (int c = 0; c < N / 16; ++c) tmem_ld16(t_lane + colA + c * 16, y + c * 16);
         tmem_wait_ld();
-        float rmax = 0.0f;
-#pragma unroll
-        for (int e = 0; e < N; ++e) rmax = fmaxf(rmax, fabsf(y[e]));
-        s_exp = prescale_exp(rmax);
+        s_exp = prescale_exp(absmax<N>(y));
         const float sc = exp2i(s_exp);
+        const float2 sc2 = make_float2(sc, sc);
+        const float2 neg1 = make_float2(-1.0f, -1.0f);
+        // each 16-column block of the row becomes 8 words of hi then 8 words of lo
 #pragma unroll
         for (int c = 0; c < N / 16; ++c) {
-          uint32_t hw[8], lw[8];
+          uint32_t hl[16];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const float a = y[c * 16 + 2 * e] * sc, b = y[c * 16 + 2 * e + 1] * sc;
-            const __half2 h = __floats2half2_rn(a, b);
-            const float2 hf = __half22float2(h);
-            hw[e] = h2_bits(h);
-            lw[e] = h2_bits(__floats2half2_rn(a - hf.x, b - hf.y));
+            const float2 v = __fmul2_rn(make_float2(y[c * 16 + 2 * e], y[c * 16 + 2 * e + 1]), sc2);
+            const __half2 h = __float22half2_rn(v);
+            const float2 r = __ffma2_rn(__half22float2(h), neg1, v);  // v - hi, exact
+            hl[e] = h2_bits(h);
+            hl[8 + e] = h2_bits(__float22half2_rn(r));
           }
-          tmem_st8(t_lane + colA + c * 8, hw);
-          tmem_st8(t_lane + colA + N / 2 + c * 8, lw);
+          tmem_st16(t_lane + colA + c * 16, hl);
         }
+        bars->srow[i & 3][row] = int8_t(s_exp);
         tmem_wait_st();
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->ys_full[g]);
+      if (lane == 0) {
+        mbar_arrive(&bars->ys_full[b]);
+        mbar_arrive(&bars->srow_full[i & 3]);
+      }
+      if (!ok) break;
+    }
+  } else {
+    // ---------------- quantizer: X'' = D * 2^crow -> codes and scales ----------------
+    setmaxnreg_inc<kHighRegs>();
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const uint32_t t_lane = tmem + (uint32_t(q * 32) << 16);
+    const bool leader = (warp == 4) && lane == 0;
+    const int tok_in_tile = row / M;
+    const int m_row = row % M;
+    int i = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
+      const int b = i & 1, j = i >> 1, ob = i & 1;
+      const uint32_t colB = uint32_t(b * 2 * N + N);
+      uint8_t* s_out = smem + G::kOffOut + ob * G::kOutStride;
+      const uint32_t s_out_u32 = sbase + G::kOffOut + ob * G::kOutStride;
+      const int64_t grow = int64_t(tile) * 128 + row;
+      const int64_t rows_left = rows_total - int64_t(tile) * 128;
+      const int valid_rows = rows_left < 128 ? int(rows_left) : 128;
+      const bool row_valid = grow < rows_total;
 
-      // ---- phase 2: X'' = D * 2^crow, quantize ----
       float d[N];
-      const bool ok2 = warp_wait(&bars->db_full[g], j & 1, bars, p.status, kStEpiBFull);
-      if (ok2) {
+      int s_exp = 0;
+      bool ok = warp_wait(&bars->db_full[b], j & 1, bars, p.status, kStEpiBFull);
+      // the splitter's row exponents of this tile. The splitter reaches tile i+4 only after
+      // this warp group has released D_B of tile i, so this wait is never more than one
+      // phase of srow_full[i % 4] behind.
+      ok = ok && warp_wait(&bars->srow_full[i & 3], (i >> 2) & 1, bars, p.status, kStEpiAFull);
+      if (ok) {
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < N / 16; ++c) tmem_ld16(t_lane + colB + c * 16, d + c * 16);
+        s_exp = bars->srow[i & 3][row];
         tmem_wait_ld();
       } else {
 #pragma unroll
@@ -535,11 +632,10 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->tm_empty[g]);
+      if (lane == 0) mbar_arrive(&bars->tm_empty[b]);
 
       const int crow = -(s_exp + t_exp);
       const float fcrow = exp2i(crow);
-      const bool row_valid = grow < rows_total;
 
       if constexpr (kMode == kModeRotate) {
         if (row_valid) {
@@ -548,54 +644,53 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
           for (int e = 0; e < N; e += 4)
             dst[e / 4] = make_float4(d[e] * fcrow, d[e + 1] * fcrow, d[e + 2] * fcrow, d[e + 3] * fcrow);
         }
-        if (leader) bars->group_exit[g] = *reinterpret_cast<volatile int*>(&bars->abort);
-        named_bar(bar_id, 128);
-        if (bars->group_exit[g]) break;
+        if (leader) bars->group_exit[ob] = *reinterpret_cast<volatile int*>(&bars->abort) | int(!ok);
+        named_bar(1, 128);
+        if (bars->group_exit[ob]) break;
         continue;
       } else {
         uint32_t words[N / 8];
         if constexpr (kMode == kModePerToken) {
-          float rmax = 0.0f;
-#pragma unroll
-          for (int e = 0; e < N; ++e) rmax = fmaxf(rmax, fabsf(d[e]));
-          const float wm = warp_max(rmax * fcrow);
-          if (lane == 0) bars->red[g][q] = wm;
-          if (leader) bulk_wait_read0();
-          named_bar(bar_id, 128);
+          const float wm = warp_max(absmax<N>(d) * fcrow);
+          if (lane == 0) bars->red[ob][q] = wm;
+          if (leader) bulk_wait_read<1>();
+          named_bar(1, 128);
           float amax = 0.0f;
           const int q0 = (tok_in_tile * M) >> 5, nq = (M + 31) >> 5;
-          for (int qq = 0; qq < nq; ++qq) amax = fmaxf(amax, bars->red[g][q0 + qq]);
+          for (int qq = 0; qq < nq; ++qq) amax = fmaxf(amax, bars->red[ob][q0 + qq]);
           const float qs = per_token_scale(amax, p.clip_ratio);
           const float inv = qs > 0.0f ? __frcp_rn(qs) : 0.0f;
           const float F = inv * fcrow;
+          const float2 F2 = make_float2(F, F);
+          const float2 magic = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
           if (row_valid && m_row == 0) p.quant_scale[grow / M] = qs;
 #pragma unroll
           for (int w = 0; w < N / 8; ++w) {
             uint32_t acc = 0u;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float v = fminf(fmaxf(d[w * 8 + e] * F, -8.0f), 7.0f);
-              acc |= (uint32_t(__float2int_rn(v)) & 0xFu) << (4 * e);
+            for (int e = 0; e < 8; e += 2) {
+              float2 v = __fmul2_rn(make_float2(d[w * 8 + e], d[w * 8 + e + 1]), F2);
+              v.x = fminf(fmaxf(v.x, -8.0f), 7.0f);
+              v.y = fminf(fmaxf(v.y, -8.0f), 7.0f);
+              // adding 1.5 * 2^23 rounds to an integer (half to even) held in the low bits
+              const float2 u = __fadd2_rn(v, magic);
+              acc = bfi4(__float_as_uint(u.x), acc, 4 * e);
+              acc = bfi4(__float_as_uint(u.y), acc, 4 * e + 4);
             }
             words[w] = acc;
           }
         } else {
-          // per-group E2M1: segment maxima over 16 columns, groups of 32 in the flattened
+          // per-group E2M1: maxima over 16-column segments, groups of 32 in the flattened
           // token; when N % 32 == 16 a row pair (2r, 2r+1) shares one group across the
           // row end, combined through a lane shuffle (the pair sits in adjacent lanes).
           constexpr int NS = N / 16;
           float smax[NS];
 #pragma unroll
-          for (int sgi = 0; sgi < NS; ++sgi) {
-            float m = 0.0f;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) m = fmaxf(m, fabsf(d[sgi * 16 + e]));
-            smax[sgi] = m;
-          }
+          for (int sgi = 0; sgi < NS; ++sgi) smax[sgi] = absmax16(d + sgi * 16);
           float Fseg[NS];
           uint8_t* s_scale = s_out + G::kCodeBytes;
-          if (leader) bulk_wait_read0();
-          named_bar(bar_id, 128);
+          if (leader) bulk_wait_read<1>();
+          named_bar(1, 128);
           if constexpr ((N % 32) == 0) {
 #pragma unroll
             for (int gi = 0; gi < NS / 2; ++gi) {
@@ -609,7 +704,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
           } else {
             constexpr int GF = (N - 16) / 32;  // full groups per row
             const bool odd = (row & 1) != 0;
-            // the straddling half-group: last 16 columns of an even row, first 16 of an odd row
+            // the straddling group: last 16 columns of an even row + first 16 of the next
             const float part = (odd ? smax[0] : smax[NS - 1]) * fcrow;
             const float other = __shfl_xor_sync(0xffffffffu, part, 1);
             const MxScale mst = mx_scale(fmaxf(part, other), p.rule);
@@ -633,12 +728,12 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
           }
 #pragma unroll
           for (int w = 0; w < N / 8; ++w) {
-            const float F = Fseg[w >> 1];
-            uint32_t acc = 0u;
-#pragma unroll
-            for (int e = 0; e < 8; e += 2)
-              acc |= e2m1x2_raw(d[w * 8 + e] * F, d[w * 8 + e + 1] * F) << (4 * e);
-            words[w] = e2m1_canonical_zero(acc);
+            const float2 F2 = make_float2(Fseg[w >> 1], Fseg[w >> 1]);
+            const float2 v0 = __fmul2_rn(make_float2(d[w * 8 + 0], d[w * 8 + 1]), F2);
+            const float2 v1 = __fmul2_rn(make_float2(d[w * 8 + 2], d[w * 8 + 3]), F2);
+            const float2 v2 = __fmul2_rn(make_float2(d[w * 8 + 4], d[w * 8 + 5]), F2);
+            const float2 v3 = __fmul2_rn(make_float2(d[w * 8 + 6], d[w * 8 + 7]), F2);
+            words[w] = e2m1_canonical_zero(e2m1x8(v0, v1, v2, v3));
           }
         }
         // codes of this row: N/2 bytes at row * N/2 in the staging buffer
@@ -652,8 +747,8 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
           for (int w = 0; w < N / 8; w += 2) dst[w / 2] = make_uint2(words[w], words[w + 1]);
         }
         fence_proxy_async();
-        if (leader) bars->group_exit[g] = *reinterpret_cast<volatile int*>(&bars->abort);
-        named_bar(bar_id, 128);
+        if (leader) bars->group_exit[ob] = *reinterpret_cast<volatile int*>(&bars->abort) | int(!ok);
+        named_bar(1, 128);
         if (leader) {
           const int64_t row0 = int64_t(tile) * 128;
           bulk_store(p.out + row0 * (N / 2), s_out_u32, uint32_t(valid_rows * (N / 2)));
@@ -661,7 +756,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
             bulk_store(p.scales + (row0 * N) / 32, s_out_u32 + G::kCodeBytes, uint32_t((valid_rows * N) / 32));
           bulk_commit();
         }
-        if (bars->group_exit[g]) break;
+        if (bars->group_exit[ob]) break;
       }
     }
     if (leader) bulk_wait_all();
@@ -669,7 +764,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, G::kTmemCols);
   }
@@ -707,7 +802,13 @@ cudaError_t launch_n(const TcParams& p, int num_sms, cudaStream_t stream) {
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
   auto kern = tc_kernel<N, kF16, kMode>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::kSmem);
+  // The register split is sized for kLaunchRegs per thread; a kernel built with fewer
+  // would make setmaxnreg.inc wait for registers that do not exist, so refuse it.
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidKernelImage;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::kSmem);
   if (e != cudaSuccess) return e;
   const int64_t tiles = (p.K * p.M + 127) / 128;
   const int grid = int(tiles < num_sms ? tiles : num_sms);
