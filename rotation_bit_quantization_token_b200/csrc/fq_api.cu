@@ -46,6 +46,7 @@ bool mx_rule_from(double d, fq::MxRule* r) {
   else if (d == 7.0) r->mode = fq::kMxMantissa7;
   else r->mode = fq::kMxRatio;
   r->dst_max = float(d);
+  r->inv_dst = d > 0.0 ? float(1.0 / d) : 0.0f;
   return true;
 }
 
@@ -152,7 +153,7 @@ fq_status fq_quantize_per_token(fq_handle* h, const void* x, const void* P1, con
   }
   if (!aligned(x, 2) || !aligned(P1, 2) || !aligned(P2, 2) || !aligned(quantScale, 4))
     return FQ_ERR_INVALID;
-  fq::MxRule rule{fq::kMxFloor, 0.0f};
+  fq::MxRule rule{fq::kMxFloor, 0.0f, 0.0f};
   return launch(h, fq::kModePerToken, x, P1, P2, clipRatio, rule, static_cast<uint8_t*>(out),
                 quantScale, nullptr, nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -177,7 +178,7 @@ fq_status fq_debug_rotate(fq_handle* h, const void* x, const void* P1, const voi
   if (h == nullptr || x == nullptr || P1 == nullptr || x2 == nullptr) return FQ_ERR_NULLPTR;
   if (!aligned(x, 2) || !aligned(P1, 2) || (P2 != nullptr && !aligned(P2, 2)) || !aligned(x2, 4))
     return FQ_ERR_INVALID;
-  fq::MxRule rule{fq::kMxFloor, 0.0f};
+  fq::MxRule rule{fq::kMxFloor, 0.0f, 0.0f};
   return launch(h, fq::kModeRotate, x, P1, P2, 1.0, rule, nullptr, nullptr, nullptr, x2,
                 reinterpret_cast<cudaStream_t>(stream));
 }

@@ -16,6 +16,7 @@ enum MxCase : int { kMxFloor = 1, kMxMantissa6 = 2, kMxMantissa7 = 3, kMxRatio =
 struct MxRule {
   int mode;        // MxCase
   float dst_max;   // float32(dstTypeMax) for the ratio rule
+  float inv_dst;   // float32(1 / dstTypeMax), used by the tensor-core kernel
 };
 
 // E8M0 byte and the exact power-of-two multiplier R such that each element of the
@@ -37,10 +38,14 @@ __device__ __forceinline__ float pow2_from_e8m0_inverse(uint32_t b) {
 //  case 3 (other):   S = fp32(amax / dstTypeMax); E = biased exponent of S, plus one
 //                    when S is normal, E < 254 and S's mantissa field is nonzero.
 // For the first two cases a zero or subnormal amax always clamps to e = -127 (byte 0).
+template <bool kExactDiv = true>
 __device__ __forceinline__ MxScale mx_scale(float amax, MxRule rule) {
   MxScale s;
   if (rule.mode == kMxRatio) {
-    const float S = __fdiv_rn(amax, rule.dst_max);
+    // S = amax / dstTypeMax in float32. The tensor-core kernel multiplies by the
+    // float32 reciprocal instead (kExactDiv = false): the product is within one ulp of
+    // the quotient, which moves the byte only when amax / dstTypeMax is a power of two.
+    const float S = kExactDiv ? __fdiv_rn(amax, rule.dst_max) : amax * rule.inv_dst;
     const uint32_t bits = __float_as_uint(S);
     uint32_t E = (bits >> 23) & 0xFFu;
     const uint32_t mant = bits & 0x7FFFFFu;

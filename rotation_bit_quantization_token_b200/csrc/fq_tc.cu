@@ -168,22 +168,6 @@ __device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
-__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
-__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    smem_u32(bar))
@@ -212,16 +196,30 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// Shared-memory matrix descriptor (tcgen05): start, leading / stride byte offsets,
-// version 1, 128-byte swizzle.
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = 0;
-  d |= uint64_t((saddr >> 4) & 0x3FFFu);
-  d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
-  d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
-  d |= uint64_t(1) << 46;
-  d |= uint64_t(2) << 61;
-  return d;
+
+// Every descriptor here shares its high word: stride byte offset 1024 (8 rows of 128 B),
+// version 1, 128-byte swizzle. The low word holds the start address (>> 4) and the
+// leading byte offset (>> 4); shared-memory addresses are below 2^18, so no masking.
+constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+__device__ __forceinline__ uint32_t desc_lo(uint32_t saddr, uint32_t lbo) { return (saddr >> 4) | ((lbo >> 4) << 16); }
+__device__ __forceinline__ void mma_ss_lo(uint32_t d, uint32_t a_lo, uint32_t b_lo, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "mov.b64 da, {%1, %5};\n\t"
+      "mov.b64 db, {%2, %5};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n\t}" ::"r"(d),
+      "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(acc), "n"(kDescHi)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_lo(uint32_t d, uint32_t a_tmem, uint32_t b_lo, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "mov.b64 db, {%2, %5};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %3, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(acc), "n"(kDescHi)
+      : "memory");
 }
 
 // Instruction descriptor, kind::f16, fp32 accumulate, M = 128.
@@ -498,13 +496,14 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
           return false;
         tc_fence_after();
         const uint32_t d = tmem + uint32_t(b * 2 * N);
-        const uint32_t xs = sbase + G::kOffX + s * G::kXStage;
+        // low descriptor words: base + a compile-time offset per MMA (about five
+        // instructions per MMA, so the issue keeps up with the tensor pipe)
+        const uint32_t a_lo = desc_lo(sbase + G::kOffP1, 16);
+        const uint32_t x_lo = desc_lo(sbase + G::kOffX + s * G::kXStage, 16384);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = sdesc(sbase + G::kOffP1 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          const uint64_t bx = sdesc(xs + kk * 2048, 16384, 1024);
-          mma_ss(d, a, bx, kIdA, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss_lo(d, a_lo + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), x_lo + ((kk * 2048) >> 4), kIdA,
+                    kk > 0 ? 1u : 0u);
         mma_commit(&bars->x_empty[s]);
         mma_commit(&bars->da_full[b]);
         return true;
@@ -516,13 +515,13 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
         tc_fence_after();
         const uint32_t d = tmem + uint32_t(b * 2 * N + N);
         const uint32_t a0 = tmem + uint32_t(b * 2 * N);
+        const uint32_t p2_lo = desc_lo(sbase + G::kOffP2, 16);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
 #pragma unroll
-          for (int kk = 0; kk < N / 16; ++kk) {
-            const uint64_t bp = sdesc(sbase + G::kOffP2 + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024);
-            mma_ts(d, a0 + uint32_t(kk * 16 + h * 8), bp, kIdB, (h | kk) != 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < N / 16; ++kk)
+            mma_ts_lo(d, a0 + uint32_t(kk * 16 + h * 8), p2_lo + (((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4),
+                      kIdB, (h | kk) != 0 ? 1u : 0u);
         }
         mma_commit(&bars->db_full[b]);
         return true;
@@ -695,7 +694,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
 #pragma unroll
             for (int gi = 0; gi < NS / 2; ++gi) {
               const float amax = fmaxf(smax[2 * gi], smax[2 * gi + 1]) * fcrow;
-              const MxScale ms = mx_scale(amax, p.rule);
+              const MxScale ms = mx_scale<false>(amax, p.rule);
               const float F = exp2i(127 - int(ms.byte) + crow);
               Fseg[2 * gi] = F;
               Fseg[2 * gi + 1] = F;
@@ -707,14 +706,14 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
             // the straddling group: last 16 columns of an even row + first 16 of the next
             const float part = (odd ? smax[0] : smax[NS - 1]) * fcrow;
             const float other = __shfl_xor_sync(0xffffffffu, part, 1);
-            const MxScale mst = mx_scale(fmaxf(part, other), p.rule);
+            const MxScale mst = mx_scale<false>(fmaxf(part, other), p.rule);
             const float Fst = exp2i(127 - int(mst.byte) + crow);
             const int pair_base = (row >> 1) * (N / 16);
             float Ff[GF];
 #pragma unroll
             for (int gi = 0; gi < GF; ++gi) {
               const float a = odd ? fmaxf(smax[2 * gi + 1], smax[2 * gi + 2]) : fmaxf(smax[2 * gi], smax[2 * gi + 1]);
-              const MxScale ms = mx_scale(a * fcrow, p.rule);
+              const MxScale ms = mx_scale<false>(a * fcrow, p.rule);
               Ff[gi] = exp2i(127 - int(ms.byte) + crow);
               s_scale[pair_base + (odd ? GF + 1 : 0) + gi] = uint8_t(ms.byte);
             }
