@@ -26,9 +26,10 @@
 //               codes, stages them in shared memory and stores them with bulk copies
 //               (double-buffered staging)
 //   warp 8      TMA producer: x tiles (128 rows x N, 128B-swizzled) into a 4-stage ring
-//   warp 9      MMA issuer: stage A (A = BD(P1) in SMEM, B = x tile, MN-major) and
-//               stage B (A = hi/lo Y in TMEM, B = P2^T in SMEM); owns the TMEM
-//   warps 10-11 idle after the prologue
+//   warps 9-10  MMA issuers, one per TMEM buffer (even / odd local tiles): stage A
+//               (A = BD(P1) in SMEM, B = x tile, MN-major) and stage B (A = hi/lo Y in
+//               TMEM, B = P2^T in SMEM); warp 9 owns the TMEM allocation
+//   warp 11     idle after the prologue
 // Two TMEM buffers (D_A for Y, D_B for X'') let stage A of tile i+2 run while the
 // quantizer still reads tile i.
 // Every wait is bounded in time; on expiry the kernel records a code in the status word,
@@ -91,7 +92,7 @@ struct Bars {
   uint64_t db_full[2];
   uint64_t tm_empty[2];
   uint64_t srow_full[4];  // row exponents of tile i published in srow[i % 4]
-  uint64_t mma_done;
+  uint64_t mma_done[2];
   uint32_t tmem_base;
   int abort;
   int group_exit[2];  // quantizer exit decision, one slot per tile parity
@@ -395,7 +396,8 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       mbar_init(&bars->tm_empty[b], 4);
     }
     for (int r = 0; r < 4; ++r) mbar_init(&bars->srow_full[r], 4);
-    mbar_init(&bars->mma_done, 1);
+    mbar_init(&bars->mma_done[0], 1);
+    mbar_init(&bars->mma_done[1], 1);
     bars->abort = 0;
     bars->group_exit[0] = bars->group_exit[1] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -479,12 +481,15 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
         }
       }
     }
-  } else if (warp == 9) {
-    // ---------------- MMA issuer ----------------
+  } else if (warp == 9 || warp == 10) {
+    // ---------------- MMA issuers, one per TMEM buffer ----------------
+    // Warp 9 issues the MMAs of the even local tiles (buffer 0), warp 10 those of the
+    // odd tiles (buffer 1), so a slow tile in one buffer does not hold up the other;
+    // the tensor pipe interleaves the two streams. A(i) may overwrite D_A[b] once B(i-2)
+    // has read its hi / lo Y; B(i) may overwrite D_B[b] once the quantizer has read the
+    // X'' of tile i-2.
     setmaxnreg_dec<kLowRegs>();
-    // Order A(i), A(i+1), B(i), B(i+1): stage A of the next pair is issued while stage B
-    // of this pair runs. A(i) may overwrite D_A[b] once B(i-2) has read its hi / lo Y;
-    // B(i) may overwrite D_B[b] once the quantizer has read the X'' of tile i-2.
+    const int mb = warp - 9;
     if (lane == 0) {
       const int n_local = (blockIdx.x < num_tiles) ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
       constexpr uint32_t kIdA = idesc_f16(!kF16, !kF16, true, N);
@@ -527,23 +532,21 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
         return true;
       };
       bool ok = true;
-      for (int i = 0; ok && i < n_local; i += 2) {
+      for (int i = mb; ok && i < n_local; i += 2) {
         ok = issue_a(i);
-        if (ok && i + 1 < n_local) ok = issue_a(i + 1);
         if (ok) ok = issue_b(i);
-        if (ok && i + 1 < n_local) ok = issue_b(i + 1);
       }
-      // every MMA issued above has completed before TMEM is released
-      mma_commit(&bars->mma_done);
-      const uint32_t b = smem_u32(&bars->mma_done);
+      // every MMA issued by this thread has completed before TMEM is released
+      mma_commit(&bars->mma_done[mb]);
+      const uint32_t b = smem_u32(&bars->mma_done[mb]);
       const uint64_t t0 = globaltimer();
       while (!mbar_try_wait(b, 0)) {
         if (globaltimer() - t0 > kTimeoutNs) { atomicOr(p.status, kStMmaDone); break; }
       }
     }
     __syncwarp();
-  } else if (warp >= 10) {
-    setmaxnreg_dec<kLowRegs>();  // idle warps of the producer / MMA warpgroup
+  } else if (warp == 11) {
+    setmaxnreg_dec<kLowRegs>();  // idle warp of the producer / MMA warpgroup
   } else if (warp < 4) {
     // ---------------- splitter: Y -> per-row power-of-two scale -> fp16 hi / lo ----------------
     setmaxnreg_inc<kHighRegs>();
