@@ -114,6 +114,34 @@ FQ_API fq_status fq_quantize_mx(fq_handle *h, const void *x, const void *P1, con
                          double dstTypeMax, void *out_fp4, uint8_t *scale_e8m0,
                          struct CUstream_st *stream);
 
+/* Per-group mode (as fq_quantize_mx) for callers that cannot allocate device memory.
+ * The paper has no counterpart: this entry point is an addition of this library.
+ *
+ * fq_create allocates a small device status block with cudaMalloc. Callers whose device
+ * memory is owned by another allocator or a fixed budget, callers that must not pay the
+ * implicit device synchronization of cudaMalloc / cudaFree on a latency-critical path,
+ * and plug-ins that may not create allocations of their own use this call instead. It
+ * takes the shape and dtype directly (no handle), allocates nothing and frees nothing:
+ * no cudaMalloc, cudaFree or allocating library routine runs in it.
+ *
+ * Its only scratch is one 32-bit status word (the word a kernel sets when one of its
+ * bounded waits gives up) inside a 256-byte static device array of the library. That
+ * array is loaded with the library's device code and held on every GPU that uses it
+ * until the process exits. Each call clears the word with cudaMemsetAsync on `stream`
+ * before the launch; the array otherwise keeps what the last call left. All calls in the
+ * process share the array, so calls that overlap on the GPU race on that word.
+ *
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ * with that device current) and caches it; make that first call before any stream
+ * capture. Arguments, layouts and errors are those of fq_quantize_mx plus the plan-phase
+ * checks of fq_create (K in [1, 262144], M, N in [1, 256], dtype): FQ_ERR_NULLPTR,
+ * FQ_ERR_INVALID (including a call whose scratch would exceed the static array, which no
+ * allowed shape does), FQ_ERR_UNSUPPORTED, FQ_ERR_CUDA. */
+FQ_API fq_status fq_quantize_mx_static(int64_t K, int64_t M, int64_t N, fq_dtype dtype,
+                                       const void *x, const void *P1, const void *P2,
+                                       double dstTypeMax, void *out_fp4, uint8_t *scale_e8m0,
+                                       struct CUstream_st *stream);
+
 /* Test hook: writes x'' = P1 . (x . P2) as float32 [K, M, N] (P2 may be NULL), computed
  * the way the selected kernel computes it before quantization. */
 FQ_API fq_status fq_debug_rotate(fq_handle *h, const void *x, const void *P1, const void *P2,

@@ -5,5 +5,6 @@ For each token of x[K, M, N]: x'' = P1 . (x . P2), quantized per token to INT4 o
 include/fq.h (libfq.so, built in-tree). The Python layer marshals arguments only.
 """
 
-from .api import FlatQuant, HostPipeline, debug_rotate, quantize_mx, quantize_per_token  # noqa: F401
+from .api import (FlatQuant, HostPipeline, debug_rotate, quantize_mx,  # noqa: F401
+                  quantize_mx_static, quantize_per_token)
 from ._lib import FQError, load as load_library  # noqa: F401

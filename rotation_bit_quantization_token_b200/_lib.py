@@ -30,6 +30,7 @@ _SIGNATURES = {
     "fq_quantize_per_token": (_int, [_vp, _vp, _vp, _vp, _dbl, _int, _vp, _vp, _vp]),
     "fq_quantize_mx": (_int, [_vp, _vp, _vp, _vp, _dbl, _vp, _vp, _vp]),
     "fq_debug_rotate": (_int, [_vp, _vp, _vp, _vp, _vp, _vp]),
+    "fq_quantize_mx_static": (_int, [_i64, _i64, _i64, _int, _vp, _vp, _vp, _dbl, _vp, _vp, _vp]),
     "fq_set_kernel": (_int, [_vp, _int]),
     "fq_last_kernel": (_int, [_vp]),
     "fq_last_launch_count": (_int, [_vp]),

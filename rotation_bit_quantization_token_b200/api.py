@@ -151,6 +151,30 @@ def quantize_mx(x, P1, P2, dst_type_max=0.0, kernel="auto"):
     return FlatQuant(K, M, N, x.dtype, kernel).quantize_mx(x, P1, P2, dst_type_max)
 
 
+def quantize_mx_static(x, P1, P2, dst_type_max=0.0, out=None, scales=None, stream=None):
+    """Per-group quantization through fq_quantize_mx_static: no handle, and the library
+    allocates nothing (its scratch is a static device array). Outputs are allocated here
+    by torch unless passed in."""
+    lib = _lib.load()
+    if x.dtype not in _DT:
+        raise ValueError("x must be bfloat16 or float16")
+    for name, t in (("x", x), ("P1", P1)):
+        _check_input(name, t, x.dtype)
+    if P2 is not None and P2.numel() == 0:
+        P2 = None
+    if P2 is not None:
+        _check_input("P2", P2, x.dtype)
+    K, M, N = x.shape
+    if out is None:
+        out = torch.empty((K, M * N // 2), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((K, -(-M * N // 64), 2), dtype=torch.uint8, device=x.device)
+    _lib.check(lib.fq_quantize_mx_static(K, M, N, _DT[x.dtype], _ptr(x), _ptr(P1), _ptr(P2),
+                                         float(dst_type_max), _ptr(out), _ptr(scales),
+                                         _stream_ptr(stream)), "fq_quantize_mx_static")
+    return out, scales
+
+
 def debug_rotate(x, P1, P2, kernel="auto"):
     K, M, N = x.shape
     return FlatQuant(K, M, N, x.dtype, kernel).debug_rotate(x, P1, P2)

@@ -95,6 +95,8 @@ fq_status launch(fq_handle* h, int mode, const void* x, const void* P1, const vo
 
 }  // namespace
 
+void fq::record_cuda_error(int e) { g_last_cuda_error = e; }
+
 extern "C" {
 
 fq_status fq_create(fq_handle** h, int64_t K, int64_t M, int64_t N, fq_dtype dtype) {

@@ -48,6 +48,9 @@ struct TcParams {
 };
 
 bool tc_supported(int64_t K, int M, int N);
+
+// Keeps a CUDA error code for fq_last_cuda_error() (thread-local).
+void record_cuda_error(int e);
 cudaError_t launch_tc(const TcParams& p, bool fp16_in, int num_sms, cudaStream_t stream);
 
 }  // namespace fq
