@@ -90,13 +90,20 @@ def load_peaks():
         return 6650.0, 1590.0, "fallback"
 
 
-def kernel_source_hash():
+KERNEL_SOURCES = {
+    "tcgen05": ["fq_tc.cu", "fq_quant.cuh", "fq_internal.h"],
+    "general": ["fq_general.cu", "fq_quant.cuh", "fq_internal.h"],
+}
+
+
+def kernel_source_hash(kernel="tcgen05"):
+    """Hash of the source files of one kernel (a recorded DRAM-traffic figure is valid only
+    for the source it was captured on)."""
     h = hashlib.sha256()
-    for name in sorted(os.listdir(CSRC)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(CSRC, name), "rb") as f:
-                h.update(name.encode())
-                h.update(f.read())
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -327,7 +334,7 @@ def run_ours(args, rank, world, local):
     bytes_per_launch = w.bytes_per_token() * K
     achieved = bytes_per_launch / (kernel_ms_max / 1e3) / 1e9
     kname = fq.last_kernel
-    src_hash = kernel_source_hash()
+    src_hash = kernel_source_hash(kname)
     traffic = recorded_traffic(kname, w.name, src_hash)
 
     # end to end through the public API: pinned host buffers, copies inside the region
