@@ -19,17 +19,18 @@
 // range, converted to fp16 and transposed to K-major once per CTA. The powers of two
 // are undone exactly in the epilogue.
 //
-// Roles (one CTA per SM, persistent over tiles, 384 threads = 3 warpgroups):
+// Roles (one CTA per SM, persistent over tiles, 512 threads = 4 warpgroups):
 //   warps 0-3   splitter: reads Y from TMEM (lane = row), scales each row by a power of
 //               two, writes fp16 hi / lo back into the same TMEM columns for stage B
-//   warps 4-7   quantizer: reads X'' from TMEM, forms per-token or per-group scales and
-//               codes, stages them in shared memory and stores them with bulk copies
-//               (double-buffered staging)
-//   warp 8      TMA producer: x tiles (128 rows x N, 128B-swizzled) into a 4-stage ring
-//   warps 9-10  MMA issuers, one per TMEM buffer (even / odd local tiles): stage A
-//               (A = BD(P1) in SMEM, B = x tile, MN-major) and stage B (A = hi/lo Y in
-//               TMEM, B = P2^T in SMEM); warp 9 owns the TMEM allocation
-//   warp 11     idle after the prologue
+//   warps 4-7   quantizer for TMEM buffer 0 (even local tiles), warps 8-11 for buffer 1
+//               (odd tiles): read a row of X'' from TMEM in one round trip, release the
+//               buffer, form per-token or per-group scales and codes, stage them in shared
+//               memory and store them with bulk copies
+//   warp 12     TMA producer: x tiles (128 rows x N, 128B-swizzled) into a 4-stage ring
+//   warps 13-14 MMA issuers, one per TMEM buffer: stage A (A = BD(P1) in SMEM, B = x tile,
+//               MN-major) and stage B (A = hi/lo Y in TMEM, B = P2^T in SMEM); warp 13
+//               owns the TMEM allocation
+//   warp 15     idle after the prologue
 // Two TMEM buffers (D_A for Y, D_B for X'') let stage A of tile i+2 run while the
 // quantizer still reads tile i.
 // Every wait is bounded in time; on expiry the kernel records a code in the status word,
@@ -49,13 +50,13 @@ namespace fq {
 namespace {
 
 constexpr int kStages = 4;
-constexpr int kThreads = 384;  // three warpgroups
-// Register split (setmaxnreg): launched at kLaunchRegs per thread; the producer / MMA
-// warpgroup drops to kLowRegs and the two epilogue warpgroups rise to kHighRegs, using
-// exactly the registers the block was launched with:
-// 2 * 128 * kHighRegs + 128 * kLowRegs == kThreads * kLaunchRegs.
-constexpr int kLaunchRegs = 168, kLowRegs = 56, kHighRegs = 224;
-static_assert(2 * 128 * kHighRegs + 128 * kLowRegs == kThreads * kLaunchRegs, "register split");
+constexpr int kThreads = 512;  // four warpgroups
+// Register split (setmaxnreg): launched at kLaunchRegs per thread; the splitter and the
+// two quantizer warpgroups rise to kSplitRegs / kQuantRegs and the producer / MMA
+// warpgroup drops to kLowRegs. The shares add up to no more than the registers the block was
+// launched with, so setmaxnreg.inc always finds what it asks for.
+constexpr int kLaunchRegs = 128, kSplitRegs = 152, kQuantRegs = 152, kLowRegs = 56;
+static_assert(128 * (kSplitRegs + 2 * kQuantRegs + kLowRegs) <= kThreads * kLaunchRegs, "register split");
 constexpr uint64_t kTimeoutNs = 4000000000ull;  // 4 s: far beyond any legitimate wait
 
 // status bits (device status word)
@@ -80,7 +81,7 @@ struct Geo {
   static constexpr int kOffX = kOffP2 + kP2Bytes;
   static constexpr int kOffOut = kOffX + kStages * kXStage;
   static constexpr int kOffBar = kOffOut + 2 * kOutStride;
-  static constexpr int kSmem = kOffBar + 1024 + 1024;       // barriers + alignment slack
+  static constexpr int kSmem = kOffBar + 4096 + 1024;       // barriers + alignment slack
   static constexpr uint32_t kTmemCols = (4 * N <= 256) ? 256u : 512u;
 };
 
@@ -95,7 +96,7 @@ struct Bars {
   uint64_t mma_done[2];
   uint32_t tmem_base;
   int abort;
-  int group_exit[2];  // quantizer exit decision, one slot per tile parity
+  int group_exit[2][2];  // per quantizer group: exit decision, one slot per use parity
   float red[2][4];
   float wmax[kThreads / 32];
   int8_t srow[4][128];  // per-row power-of-two exponent of Y, ring of four tiles
@@ -307,6 +308,20 @@ template <int n>
 __device__ __forceinline__ void setmaxnreg_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(n));
 }
+// v - float(h) for both halves, exact (h is v rounded to fp16), with one mixed-precision
+// FMA per half: h * (-1) + v, the fp16 operand widened inside the FMA.
+__device__ __forceinline__ float2 residual2(__half2 h, float2 v) {
+  float2 r;
+  const uint32_t hb = *reinterpret_cast<uint32_t*>(&h);
+  asm("{\n\t.reg .b16 lo, hi, m1;\n\t"
+      "mov.b32 {lo, hi}, %2;\n\t"
+      "mov.b16 m1, 0xBC00;\n\t"  // -1.0 in fp16
+      "fma.rn.f32.f16 %0, lo, m1, %3;\n\t"
+      "fma.rn.f32.f16 %1, hi, m1, %4;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "r"(hb), "f"(v.x), "f"(v.y));
+  return r;
+}
 // Bounded wait on an mbarrier phase. On expiry sets the abort flag and a status bit.
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, Bars* bars, uint32_t* status,
                                           uint32_t code) {
@@ -399,7 +414,8 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     mbar_init(&bars->mma_done[0], 1);
     mbar_init(&bars->mma_done[1], 1);
     bars->abort = 0;
-    bars->group_exit[0] = bars->group_exit[1] = 0;
+    bars->group_exit[0][0] = bars->group_exit[0][1] = 0;
+    bars->group_exit[1][0] = bars->group_exit[1][1] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -447,13 +463,13 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     }
   }
   fence_proxy_async();
-  if (warp == 9) tmem_alloc(&bars->tmem_base, G::kTmemCols);
+  if (warp == 13) tmem_alloc(&bars->tmem_base, G::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == 8) {
+  if (warp == 12) {
     // ---------------- TMA producer ----------------
     setmaxnreg_dec<kLowRegs>();
     if (lane == 0) {
@@ -481,7 +497,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
         }
       }
     }
-  } else if (warp == 9 || warp == 10) {
+  } else if (warp == 13 || warp == 14) {
     // ---------------- MMA issuers, one per TMEM buffer ----------------
     // Warp 9 issues the MMAs of the even local tiles (buffer 0), warp 10 those of the
     // odd tiles (buffer 1), so a slow tile in one buffer does not hold up the other;
@@ -489,7 +505,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     // has read its hi / lo Y; B(i) may overwrite D_B[b] once the quantizer has read the
     // X'' of tile i-2.
     setmaxnreg_dec<kLowRegs>();
-    const int mb = warp - 9;
+    const int mb = warp - 13;
     if (lane == 0) {
       const int n_local = (blockIdx.x < num_tiles) ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
       constexpr uint32_t kIdA = idesc_f16(!kF16, !kF16, true, N);
@@ -545,11 +561,11 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       }
     }
     __syncwarp();
-  } else if (warp == 11) {
+  } else if (warp == 15) {
     setmaxnreg_dec<kLowRegs>();  // idle warp of the producer / MMA warpgroup
   } else if (warp < 4) {
     // ---------------- splitter: Y -> per-row power-of-two scale -> fp16 hi / lo ----------------
-    setmaxnreg_inc<kHighRegs>();
+    setmaxnreg_inc<kSplitRegs>();
     const int q = warp & 3;
     const int row = q * 32 + lane;
     const uint32_t t_lane = tmem + (uint32_t(q * 32) << 16);
@@ -569,7 +585,6 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
         s_exp = prescale_exp(absmax<N>(y));
         const float sc = exp2i(s_exp);
         const float2 sc2 = make_float2(sc, sc);
-        const float2 neg1 = make_float2(-1.0f, -1.0f);
         // each 16-column block of the row becomes 8 words of hi then 8 words of lo
 #pragma unroll
         for (int c = 0; c < N / 16; ++c) {
@@ -578,9 +593,8 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
           for (int e = 0; e < 8; ++e) {
             const float2 v = __fmul2_rn(make_float2(y[c * 16 + 2 * e], y[c * 16 + 2 * e + 1]), sc2);
             const __half2 h = __float22half2_rn(v);
-            const float2 r = __ffma2_rn(__half22float2(h), neg1, v);  // v - hi, exact
             hl[e] = h2_bits(h);
-            hl[8 + e] = h2_bits(__float22half2_rn(r));
+            hl[8 + e] = h2_bits(__float22half2_rn(residual2(h, v)));
           }
           tmem_st16(t_lane + colA + c * 16, hl);
         }
@@ -596,36 +610,43 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       if (!ok) break;
     }
   } else {
-    // ---------------- quantizer: X'' = D * 2^crow -> codes and scales ----------------
-    setmaxnreg_inc<kHighRegs>();
+    // ---------------- quantizers: X'' = D * 2^crow -> codes and scales ----------------
+    // Two warpgroups, one per TMEM buffer (even / odd local tiles). A thread reads its whole
+    // row of X'' in one TMEM round trip and releases the buffer at once, so stage B of tile
+    // i+2 can start while tile i is still being encoded.
+    setmaxnreg_inc<kQuantRegs>();
+    const int qb = (warp >> 2) - 1;        // TMEM buffer and staging buffer of this group
     const int q = warp & 3;
     const int row = q * 32 + lane;
     const uint32_t t_lane = tmem + (uint32_t(q * 32) << 16);
-    const bool leader = (warp == 4) && lane == 0;
+    const uint32_t colB = uint32_t(qb * 2 * N + N);
+    const bool leader = (q == 0) && lane == 0;
+    const int bar_id = 1 + qb;
     const int tok_in_tile = row / M;
     const int m_row = row % M;
-    int i = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
-      const int b = i & 1, j = i >> 1, ob = i & 1;
-      const uint32_t colB = uint32_t(b * 2 * N + N);
-      uint8_t* s_out = smem + G::kOffOut + ob * G::kOutStride;
-      const uint32_t s_out_u32 = sbase + G::kOffOut + ob * G::kOutStride;
+    uint8_t* s_out = smem + G::kOffOut + qb * G::kOutStride;
+    const uint32_t s_out_u32 = sbase + G::kOffOut + qb * G::kOutStride;
+    constexpr int NS = N / 16;                 // 16-column segments
+
+    int jj = 0;  // use count of this buffer
+    for (int i = qb, tile = blockIdx.x + qb * gridDim.x; tile < num_tiles;
+         i += 2, tile += 2 * gridDim.x, ++jj) {
       const int64_t grow = int64_t(tile) * 128 + row;
       const int64_t rows_left = rows_total - int64_t(tile) * 128;
       const int valid_rows = rows_left < 128 ? int(rows_left) : 128;
       const bool row_valid = grow < rows_total;
 
+      bool ok = warp_wait(&bars->db_full[qb], jj & 1, bars, p.status, kStEpiBFull);
+      // the splitter's row exponents of this tile. The splitter reaches tile i+4 only after
+      // this group has released D_B of tile i, so this wait is never more than one phase
+      // of srow_full[i % 4] behind.
+      ok = ok && warp_wait(&bars->srow_full[i & 3], (i >> 2) & 1, bars, p.status, kStEpiAFull);
       float d[N];
       int s_exp = 0;
-      bool ok = warp_wait(&bars->db_full[b], j & 1, bars, p.status, kStEpiBFull);
-      // the splitter's row exponents of this tile. The splitter reaches tile i+4 only after
-      // this warp group has released D_B of tile i, so this wait is never more than one
-      // phase of srow_full[i % 4] behind.
-      ok = ok && warp_wait(&bars->srow_full[i & 3], (i >> 2) & 1, bars, p.status, kStEpiAFull);
       if (ok) {
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < N / 16; ++c) tmem_ld16(t_lane + colB + c * 16, d + c * 16);
+        for (int c = 0; c < NS; ++c) tmem_ld16(t_lane + colB + c * 16, d + c * 16);
         s_exp = bars->srow[i & 3][row];
         tmem_wait_ld();
       } else {
@@ -634,8 +655,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->tm_empty[b]);
-
+      if (lane == 0) mbar_arrive(&bars->tm_empty[qb]);
       const int crow = -(s_exp + t_exp);
       const float fcrow = exp2i(crow);
 
@@ -646,67 +666,48 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
           for (int e = 0; e < N; e += 4)
             dst[e / 4] = make_float4(d[e] * fcrow, d[e + 1] * fcrow, d[e + 2] * fcrow, d[e + 3] * fcrow);
         }
-        if (leader) bars->group_exit[ob] = *reinterpret_cast<volatile int*>(&bars->abort) | int(!ok);
-        named_bar(1, 128);
-        if (bars->group_exit[ob]) break;
+        if (leader) bars->group_exit[qb][jj & 1] = *reinterpret_cast<volatile int*>(&bars->abort) | int(!ok);
+        named_bar(bar_id, 128);
+        if (bars->group_exit[qb][jj & 1]) break;
         continue;
       } else {
-        uint32_t words[N / 8];
+        float smax[NS];
+#pragma unroll
+        for (int sg = 0; sg < NS; ++sg) smax[sg] = absmax16(d + sg * 16);
+        if (leader) bulk_wait_read<0>();  // this group's previous store has left the staging buffer
+        float Fseg[NS];
         if constexpr (kMode == kModePerToken) {
-          const float wm = warp_max(absmax<N>(d) * fcrow);
-          if (lane == 0) bars->red[ob][q] = wm;
-          if (leader) bulk_wait_read<1>();
-          named_bar(1, 128);
+          float rmax = 0.0f;
+#pragma unroll
+          for (int sg = 0; sg < NS; ++sg) rmax = fmaxf(rmax, smax[sg]);
+          const float wm = warp_max(rmax * fcrow);
+          if (lane == 0) bars->red[qb][q] = wm;
+          named_bar(bar_id, 128);
           float amax = 0.0f;
           const int q0 = (tok_in_tile * M) >> 5, nq = (M + 31) >> 5;
-          for (int qq = 0; qq < nq; ++qq) amax = fmaxf(amax, bars->red[ob][q0 + qq]);
+          for (int qq = 0; qq < nq; ++qq) amax = fmaxf(amax, bars->red[qb][q0 + qq]);
           const float qs = per_token_scale(amax, p.clip_ratio);
           const float inv = qs > 0.0f ? __frcp_rn(qs) : 0.0f;
-          const float F = inv * fcrow;
-          const float2 F2 = make_float2(F, F);
-          const float2 magic = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
           if (row_valid && m_row == 0) p.quant_scale[grow / M] = qs;
 #pragma unroll
-          for (int w = 0; w < N / 8; ++w) {
-            uint32_t acc = 0u;
-#pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-              float2 v = __fmul2_rn(make_float2(d[w * 8 + e], d[w * 8 + e + 1]), F2);
-              v.x = fminf(fmaxf(v.x, -8.0f), 7.0f);
-              v.y = fminf(fmaxf(v.y, -8.0f), 7.0f);
-              // adding 1.5 * 2^23 rounds to an integer (half to even) held in the low bits
-              const float2 u = __fadd2_rn(v, magic);
-              acc = bfi4(__float_as_uint(u.x), acc, 4 * e);
-              acc = bfi4(__float_as_uint(u.y), acc, 4 * e + 4);
-            }
-            words[w] = acc;
-          }
+          for (int sg = 0; sg < NS; ++sg) Fseg[sg] = inv * fcrow;
         } else {
-          // per-group E2M1: maxima over 16-column segments, groups of 32 in the flattened
-          // token; when N % 32 == 16 a row pair (2r, 2r+1) shares one group across the
-          // row end, combined through a lane shuffle (the pair sits in adjacent lanes).
-          constexpr int NS = N / 16;
-          float smax[NS];
-#pragma unroll
-          for (int sgi = 0; sgi < NS; ++sgi) smax[sgi] = absmax16(d + sgi * 16);
-          float Fseg[NS];
+          named_bar(bar_id, 128);
           uint8_t* s_scale = s_out + G::kCodeBytes;
-          if (leader) bulk_wait_read<1>();
-          named_bar(1, 128);
           if constexpr ((N % 32) == 0) {
 #pragma unroll
             for (int gi = 0; gi < NS / 2; ++gi) {
-              const float amax = fmaxf(smax[2 * gi], smax[2 * gi + 1]) * fcrow;
-              const MxScale ms = mx_scale<false>(amax, p.rule);
+              const MxScale ms = mx_scale<false>(fmaxf(smax[2 * gi], smax[2 * gi + 1]) * fcrow, p.rule);
               const float F = exp2i(127 - int(ms.byte) + crow);
               Fseg[2 * gi] = F;
               Fseg[2 * gi + 1] = F;
               s_scale[row * (N / 32) + gi] = uint8_t(ms.byte);
             }
           } else {
+            // groups of 32 straddle rows: the last 16 columns of an even row and the first
+            // 16 of the next row form one group (the pair sits in adjacent lanes)
             constexpr int GF = (N - 16) / 32;  // full groups per row
             const bool odd = (row & 1) != 0;
-            // the straddling group: last 16 columns of an even row + first 16 of the next
             const float part = (odd ? smax[0] : smax[NS - 1]) * fcrow;
             const float other = __shfl_xor_sync(0xffffffffu, part, 1);
             const MxScale mst = mx_scale<false>(fmaxf(part, other), p.rule);
@@ -722,35 +723,48 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
             }
             if (!odd) s_scale[pair_base + GF] = uint8_t(mst.byte);
 #pragma unroll
-            for (int sgi = 0; sgi < NS; ++sgi) {
-              const float fe = (sgi == NS - 1) ? Fst : Ff[sgi >> 1];
-              const float fo = (sgi == 0) ? Fst : Ff[(sgi - 1) >> 1];
-              Fseg[sgi] = odd ? fo : fe;
+            for (int sg = 0; sg < NS; ++sg) {
+              const float fe = (sg == NS - 1) ? Fst : Ff[sg >> 1];
+              const float fo = (sg == 0) ? Fst : Ff[(sg - 1) >> 1];
+              Fseg[sg] = odd ? fo : fe;
             }
           }
-#pragma unroll
-          for (int w = 0; w < N / 8; ++w) {
-            const float2 F2 = make_float2(Fseg[w >> 1], Fseg[w >> 1]);
-            const float2 v0 = __fmul2_rn(make_float2(d[w * 8 + 0], d[w * 8 + 1]), F2);
-            const float2 v1 = __fmul2_rn(make_float2(d[w * 8 + 2], d[w * 8 + 3]), F2);
-            const float2 v2 = __fmul2_rn(make_float2(d[w * 8 + 4], d[w * 8 + 5]), F2);
-            const float2 v3 = __fmul2_rn(make_float2(d[w * 8 + 6], d[w * 8 + 7]), F2);
-            words[w] = e2m1_canonical_zero(e2m1x8(v0, v1, v2, v3));
-          }
         }
-        // codes of this row: N/2 bytes at row * N/2 in the staging buffer
-        if constexpr ((N % 32) == 0) {
-          uint4* dst = reinterpret_cast<uint4*>(s_out + row * (N / 2));
+        // codes: 16 columns (2 words) at a time into the staging buffer
 #pragma unroll
-          for (int w = 0; w < N / 8; w += 4) dst[w / 4] = make_uint4(words[w], words[w + 1], words[w + 2], words[w + 3]);
-        } else {
-          uint2* dst = reinterpret_cast<uint2*>(s_out + row * (N / 2));
+        for (int sg = 0; sg < NS; ++sg) {
+          const float2 F2 = make_float2(Fseg[sg], Fseg[sg]);
+          uint32_t words[2];
 #pragma unroll
-          for (int w = 0; w < N / 8; w += 2) dst[w / 2] = make_uint2(words[w], words[w + 1]);
+          for (int wd = 0; wd < 2; ++wd) {
+            const float* w = d + sg * 16 + wd * 8;
+            if constexpr (kMode == kModePerToken) {
+              const float2 magic = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+              uint32_t acc = 0u;
+#pragma unroll
+              for (int e = 0; e < 8; e += 2) {
+                float2 t = __fmul2_rn(make_float2(w[e], w[e + 1]), F2);
+                t.x = fminf(fmaxf(t.x, -8.0f), 7.0f);
+                t.y = fminf(fmaxf(t.y, -8.0f), 7.0f);
+                // adding 1.5 * 2^23 rounds to an integer (half to even) held in the low bits
+                const float2 u = __fadd2_rn(t, magic);
+                acc = bfi4(__float_as_uint(u.x), acc, 4 * e);
+                acc = bfi4(__float_as_uint(u.y), acc, 4 * e + 4);
+              }
+              words[wd] = acc;
+            } else {
+              const float2 a = __fmul2_rn(make_float2(w[0], w[1]), F2);
+              const float2 b = __fmul2_rn(make_float2(w[2], w[3]), F2);
+              const float2 cc = __fmul2_rn(make_float2(w[4], w[5]), F2);
+              const float2 dd = __fmul2_rn(make_float2(w[6], w[7]), F2);
+              words[wd] = e2m1_canonical_zero(e2m1x8(a, b, cc, dd));
+            }
+          }
+          *reinterpret_cast<uint2*>(s_out + row * (N / 2) + sg * 8) = make_uint2(words[0], words[1]);
         }
         fence_proxy_async();
-        if (leader) bars->group_exit[ob] = *reinterpret_cast<volatile int*>(&bars->abort) | int(!ok);
-        named_bar(1, 128);
+        if (leader) bars->group_exit[qb][jj & 1] = *reinterpret_cast<volatile int*>(&bars->abort) | int(!ok);
+        named_bar(bar_id, 128);
         if (leader) {
           const int64_t row0 = int64_t(tile) * 128;
           bulk_store(p.out + row0 * (N / 2), s_out_u32, uint32_t(valid_rows * (N / 2)));
@@ -758,7 +772,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
             bulk_store(p.scales + (row0 * N) / 32, s_out_u32 + G::kCodeBytes, uint32_t((valid_rows * N) / 32));
           bulk_commit();
         }
-        if (bars->group_exit[ob]) break;
+        if (bars->group_exit[qb][jj & 1]) break;
       }
     }
     if (leader) bulk_wait_all();
@@ -766,7 +780,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, G::kTmemCols);
   }
