@@ -82,24 +82,27 @@ struct Geo {
   static constexpr int kOffOut = kOffX + kStages * kXStage;
   static constexpr int kOffBar = kOffOut + 2 * kOutStride;
   static constexpr int kSmem = kOffBar + 4096 + 1024;       // barriers + alignment slack
-  static constexpr uint32_t kTmemCols = (4 * N <= 256) ? 256u : 512u;
+  // TMEM buffers of (D_A, D_B), 2N columns each: four when they fit (N = 64), else two.
+  static constexpr int kNbuf = (8 * N <= 512) ? 4 : 2;
+  static constexpr int kRing = 2 * kNbuf;  // row-exponent ring (see the quantizer)
+  static constexpr uint32_t kTmemCols = (kNbuf * 2 * N <= 256) ? 256u : 512u;
 };
 
 struct Bars {
   uint64_t x_full[kStages];
   uint64_t x_empty[kStages];
-  uint64_t da_full[2];
-  uint64_t ys_full[2];
-  uint64_t db_full[2];
-  uint64_t tm_empty[2];
-  uint64_t srow_full[4];  // row exponents of tile i published in srow[i % 4]
+  uint64_t da_full[4];
+  uint64_t ys_full[4];
+  uint64_t db_full[4];
+  uint64_t tm_empty[4];
+  uint64_t srow_full[8];  // row exponents of tile i published in srow[i % ring]
   uint64_t mma_done[2];
   uint32_t tmem_base;
   int abort;
   int group_exit[2][2];  // per quantizer group: exit decision, one slot per use parity
   float red[2][4];
   float wmax[kThreads / 32];
-  int8_t srow[4][128];  // per-row power-of-two exponent of Y, ring of four tiles
+  int8_t srow[8][128];  // per-row power-of-two exponent of Y, ring of 2 * buffers tiles
 };
 
 // ------------------------------------------------------------------------------------
@@ -404,13 +407,13 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       mbar_init(&bars->x_full[s], 1);
       mbar_init(&bars->x_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < 4; ++b) {
       mbar_init(&bars->da_full[b], 1);
       mbar_init(&bars->ys_full[b], 4);
       mbar_init(&bars->db_full[b], 1);
       mbar_init(&bars->tm_empty[b], 4);
     }
-    for (int r = 0; r < 4; ++r) mbar_init(&bars->srow_full[r], 4);
+    for (int r = 0; r < 8; ++r) mbar_init(&bars->srow_full[r], 4);
     mbar_init(&bars->mma_done[0], 1);
     mbar_init(&bars->mma_done[1], 1);
     bars->abort = 0;
@@ -498,12 +501,12 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       }
     }
   } else if (warp == 13 || warp == 14) {
-    // ---------------- MMA issuers, one per TMEM buffer ----------------
-    // Warp 9 issues the MMAs of the even local tiles (buffer 0), warp 10 those of the
-    // odd tiles (buffer 1), so a slow tile in one buffer does not hold up the other;
-    // the tensor pipe interleaves the two streams. A(i) may overwrite D_A[b] once B(i-2)
-    // has read its hi / lo Y; B(i) may overwrite D_B[b] once the quantizer has read the
-    // X'' of tile i-2.
+    // ---------------- MMA issuers ----------------
+    // Warp 13 issues the MMAs of the even local tiles, warp 14 those of the odd tiles, so a
+    // slow tile on one side does not hold up the other; the tensor pipe interleaves the
+    // two streams. Tile i uses TMEM buffer i % NB. A(i) may overwrite D_A once B(i-NB) has
+    // read its hi / lo Y; B(i) may overwrite D_B once the quantizer has read the X'' of
+    // tile i-NB. With four buffers each issuer runs stage A one of its tiles ahead.
     setmaxnreg_dec<kLowRegs>();
     const int mb = warp - 13;
     if (lane == 0) {
@@ -511,9 +514,9 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       constexpr uint32_t kIdA = idesc_f16(!kF16, !kF16, true, N);
       constexpr uint32_t kIdB = idesc_f16(false, false, false, N);
       auto issue_a = [&](int i) -> bool {
-        const int s = i % kStages, b = i & 1, j = i >> 1;
+        const int s = i % kStages, b = i % G::kNbuf, u = i / G::kNbuf;
         if (!wait_bounded(&bars->x_full[s], (i / kStages) & 1, bars, p.status, kStMmaXFull)) return false;
-        if (j >= 1 && !wait_bounded(&bars->db_full[b], (j - 1) & 1, bars, p.status, kStMmaTmemEmpty))
+        if (u >= 1 && !wait_bounded(&bars->db_full[b], (u - 1) & 1, bars, p.status, kStMmaTmemEmpty))
           return false;
         tc_fence_after();
         const uint32_t d = tmem + uint32_t(b * 2 * N);
@@ -530,9 +533,9 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
         return true;
       };
       auto issue_b = [&](int i) -> bool {
-        const int b = i & 1, j = i >> 1;
-        if (!wait_bounded(&bars->ys_full[b], j & 1, bars, p.status, kStMmaYsFull)) return false;
-        if (!wait_bounded(&bars->tm_empty[b], (j & 1) ^ 1, bars, p.status, kStMmaTmemEmpty)) return false;
+        const int b = i % G::kNbuf, u = i / G::kNbuf;
+        if (!wait_bounded(&bars->ys_full[b], u & 1, bars, p.status, kStMmaYsFull)) return false;
+        if (!wait_bounded(&bars->tm_empty[b], (u & 1) ^ 1, bars, p.status, kStMmaTmemEmpty)) return false;
         tc_fence_after();
         const uint32_t d = tmem + uint32_t(b * 2 * N + N);
         const uint32_t a0 = tmem + uint32_t(b * 2 * N);
@@ -547,9 +550,12 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
         mma_commit(&bars->db_full[b]);
         return true;
       };
+      constexpr int kAhead = G::kNbuf / 2 - 1;  // stage-A lookahead, in this issuer's tiles
       bool ok = true;
+      for (int k = 0; ok && k < kAhead; ++k)
+        if (mb + 2 * k < n_local) ok = issue_a(mb + 2 * k);
       for (int i = mb; ok && i < n_local; i += 2) {
-        ok = issue_a(i);
+        if (i + 2 * kAhead < n_local) ok = issue_a(i + 2 * kAhead);
         if (ok) ok = issue_b(i);
       }
       // every MMA issued by this thread has completed before TMEM is released
@@ -571,10 +577,10 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     const uint32_t t_lane = tmem + (uint32_t(q * 32) << 16);
     int i = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
-      const int b = i & 1, j = i >> 1;
+      const int b = i % G::kNbuf, u = i / G::kNbuf;
       const uint32_t colA = uint32_t(b * 2 * N);
       int s_exp = 0;
-      const bool ok = warp_wait(&bars->da_full[b], j & 1, bars, p.status, kStEpiAFull);
+      const bool ok = warp_wait(&bars->da_full[b], u & 1, bars, p.status, kStEpiAFull);
       if (ok) {
         tc_fence_after();
         // one TMEM round trip: the whole row, then the row maximum as a shallow tree
@@ -598,28 +604,27 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
           }
           tmem_st16(t_lane + colA + c * 16, hl);
         }
-        bars->srow[i & 3][row] = int8_t(s_exp);
+        bars->srow[i % G::kRing][row] = int8_t(s_exp);
         tmem_wait_st();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&bars->ys_full[b]);
-        mbar_arrive(&bars->srow_full[i & 3]);
+        mbar_arrive(&bars->srow_full[i % G::kRing]);
       }
       if (!ok) break;
     }
   } else {
     // ---------------- quantizers: X'' = D * 2^crow -> codes and scales ----------------
-    // Two warpgroups, one per TMEM buffer (even / odd local tiles). A thread reads its whole
+    // Two warpgroups, for the even and the odd local tiles. A thread reads its whole
     // row of X'' in one TMEM round trip and releases the buffer at once, so stage B of tile
     // i+2 can start while tile i is still being encoded.
     setmaxnreg_inc<kQuantRegs>();
-    const int qb = (warp >> 2) - 1;        // TMEM buffer and staging buffer of this group
+    const int qb = (warp >> 2) - 1;        // tile parity and staging buffer of this group
     const int q = warp & 3;
     const int row = q * 32 + lane;
     const uint32_t t_lane = tmem + (uint32_t(q * 32) << 16);
-    const uint32_t colB = uint32_t(qb * 2 * N + N);
     const bool leader = (q == 0) && lane == 0;
     const int bar_id = 1 + qb;
     const int tok_in_tile = row / M;
@@ -636,18 +641,22 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       const int valid_rows = rows_left < 128 ? int(rows_left) : 128;
       const bool row_valid = grow < rows_total;
 
-      bool ok = warp_wait(&bars->db_full[qb], jj & 1, bars, p.status, kStEpiBFull);
-      // the splitter's row exponents of this tile. The splitter reaches tile i+4 only after
-      // this group has released D_B of tile i, so this wait is never more than one phase
-      // of srow_full[i % 4] behind.
-      ok = ok && warp_wait(&bars->srow_full[i & 3], (i >> 2) & 1, bars, p.status, kStEpiAFull);
+      const int b = i % G::kNbuf, u = i / G::kNbuf;
+      const uint32_t colB = uint32_t(b * 2 * N + N);
+      bool ok = warp_wait(&bars->db_full[b], u & 1, bars, p.status, kStEpiBFull);
+      // the splitter's row exponents of this tile, in slot i % ring (ring = 2 NB). The
+      // splitter reaches tile i + ring only after this group has released D_B of tile i
+      // (A(i+ring) needs B(i+NB), which needs that release), so this wait is never more
+      // than one phase of srow_full[i % ring] behind, and the slot is not overwritten
+      // before it is read.
+      ok = ok && warp_wait(&bars->srow_full[i % G::kRing], (i / G::kRing) & 1, bars, p.status, kStEpiAFull);
       float d[N];
       int s_exp = 0;
       if (ok) {
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < NS; ++c) tmem_ld16(t_lane + colB + c * 16, d + c * 16);
-        s_exp = bars->srow[i & 3][row];
+        s_exp = bars->srow[i % G::kRing][row];
         tmem_wait_ld();
       } else {
 #pragma unroll
@@ -655,7 +664,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->tm_empty[qb]);
+      if (lane == 0) mbar_arrive(&bars->tm_empty[b]);
       const int crow = -(s_exp + t_exp);
       const float fcrow = exp2i(crow);
 
