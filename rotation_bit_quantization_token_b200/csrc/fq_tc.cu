@@ -85,6 +85,8 @@ struct Geo {
   // TMEM buffers of (D_A, D_B), 2N columns each: four when they fit (N = 64), else two.
   static constexpr int kNbuf = (8 * N <= 512) ? 4 : 2;
   static constexpr int kRing = 2 * kNbuf;  // row-exponent ring (see the quantizer)
+  static constexpr int kBlocks = N / 16;          // 16-column blocks of a row
+  static constexpr int kGroups = (kBlocks + 1) / 2;  // published two blocks at a time
   static constexpr uint32_t kTmemCols = (kNbuf * 2 * N <= 256) ? 256u : 512u;
 };
 
@@ -92,7 +94,7 @@ struct Bars {
   uint64_t x_full[kStages];
   uint64_t x_empty[kStages];
   uint64_t da_full[4];
-  uint64_t ys_full[4];
+  uint64_t ys_full[4][4];  // per buffer: hi / lo of column group g (two 16-column blocks) written
   uint64_t db_full[4];
   uint64_t tm_empty[4];
   uint64_t srow_full[8];  // row exponents of tile i published in srow[i % ring]
@@ -409,7 +411,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     }
     for (int b = 0; b < 4; ++b) {
       mbar_init(&bars->da_full[b], 1);
-      mbar_init(&bars->ys_full[b], 4);
+      for (int g = 0; g < 4; ++g) mbar_init(&bars->ys_full[b][g], 4);
       mbar_init(&bars->db_full[b], 1);
       mbar_init(&bars->tm_empty[b], 4);
     }
@@ -534,18 +536,23 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       };
       auto issue_b = [&](int i) -> bool {
         const int b = i % G::kNbuf, u = i / G::kNbuf;
-        if (!wait_bounded(&bars->ys_full[b], u & 1, bars, p.status, kStMmaYsFull)) return false;
         if (!wait_bounded(&bars->tm_empty[b], (u & 1) ^ 1, bars, p.status, kStMmaTmemEmpty)) return false;
-        tc_fence_after();
         const uint32_t d = tmem + uint32_t(b * 2 * N + N);
         const uint32_t a0 = tmem + uint32_t(b * 2 * N);
         const uint32_t p2_lo = desc_lo(sbase + G::kOffP2, 16);
+        // K-steps are issued as the splitter publishes each pair of 16-column blocks, so
+        // stage B runs alongside the split instead of after it
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int g = 0; g < G::kGroups; ++g) {
+          if (!wait_bounded(&bars->ys_full[b][g], u & 1, bars, p.status, kStMmaYsFull)) return false;
+          tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < N / 16; ++kk)
-            mma_ts_lo(d, a0 + uint32_t(kk * 16 + h * 8), p2_lo + (((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4),
-                      kIdB, (h | kk) != 0 ? 1u : 0u);
+          for (int kk = 2 * g; kk < 2 * g + 2 && kk < G::kBlocks; ++kk) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              mma_ts_lo(d, a0 + uint32_t(kk * 16 + h * 8), p2_lo + (((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4),
+                        kIdB, (h | kk) != 0 ? 1u : 0u);
+          }
         }
         mma_commit(&bars->db_full[b]);
         return true;
@@ -591,28 +598,36 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
         s_exp = prescale_exp(absmax<N>(y));
         const float sc = exp2i(s_exp);
         const float2 sc2 = make_float2(sc, sc);
-        // each 16-column block of the row becomes 8 words of hi then 8 words of lo
-#pragma unroll
-        for (int c = 0; c < N / 16; ++c) {
-          uint32_t hl[16];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float2 v = __fmul2_rn(make_float2(y[c * 16 + 2 * e], y[c * 16 + 2 * e + 1]), sc2);
-            const __half2 h = __float22half2_rn(v);
-            hl[e] = h2_bits(h);
-            hl[8 + e] = h2_bits(__float22half2_rn(residual2(h, v)));
-          }
-          tmem_st16(t_lane + colA + c * 16, hl);
-        }
         bars->srow[i % G::kRing][row] = int8_t(s_exp);
-        tmem_wait_st();
+        // each 16-column block of the row becomes 8 words of hi then 8 words of lo; every
+        // pair of blocks is published on its own barrier as soon as it is in TMEM
+#pragma unroll
+        for (int g = 0; g < G::kGroups; ++g) {
+#pragma unroll
+          for (int c = 2 * g; c < 2 * g + 2 && c < G::kBlocks; ++c) {
+            uint32_t hl[16];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float2 v = __fmul2_rn(make_float2(y[c * 16 + 2 * e], y[c * 16 + 2 * e + 1]), sc2);
+              const __half2 h = __float22half2_rn(v);
+              hl[e] = h2_bits(h);
+              hl[8 + e] = h2_bits(__float22half2_rn(residual2(h, v)));
+            }
+            tmem_st16(t_lane + colA + c * 16, hl);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->ys_full[b][g]);
+        }
+      } else {
+        // a failed wait still publishes every group, so the MMA issuer is not left waiting
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0)
+          for (int g = 0; g < G::kGroups; ++g) mbar_arrive(&bars->ys_full[b][g]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bars->ys_full[b]);
-        mbar_arrive(&bars->srow_full[i % G::kRing]);
-      }
+      if (lane == 0) mbar_arrive(&bars->srow_full[i % G::kRing]);
       if (!ok) break;
     }
   } else {
