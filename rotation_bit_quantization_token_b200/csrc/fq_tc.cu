@@ -20,19 +20,19 @@
 // are undone exactly in the epilogue.
 //
 // Roles (one CTA per SM, persistent over tiles, 512 threads = 4 warpgroups):
-//   warps 0-3   splitter: reads Y from TMEM (lane = row), scales each row by a power of
-//               two, writes fp16 hi / lo back into the same TMEM columns for stage B
-//   warps 4-7   quantizer for TMEM buffer 0 (even local tiles), warps 8-11 for buffer 1
-//               (odd tiles): read a row of X'' from TMEM in one round trip, release the
-//               buffer, form per-token or per-group scales and codes, stage them in shared
-//               memory and store them with bulk copies
+//   warps 0-11  three epilogue warpgroups; group g takes the local tiles i = g (mod 3):
+//               it reads Y from TMEM (lane = row), scales each row by a power of two and
+//               writes fp16 hi / lo back into the same TMEM columns for stage B; then it
+//               reads the row of X'' in one round trip, releases the buffer, forms
+//               per-token or per-group scales and codes, stages them in shared memory and
+//               stores them with bulk copies
 //   warp 12     TMA producer: x tiles (128 rows x N, 128B-swizzled) into a 4-stage ring
-//   warps 13-14 MMA issuers, one per TMEM buffer: stage A (A = BD(P1) in SMEM, B = x tile,
-//               MN-major) and stage B (A = hi/lo Y in TMEM, B = P2^T in SMEM); warp 13
-//               owns the TMEM allocation
+//   warp 13     MMA issuer of stage A (A = BD(P1) in SMEM, B = x tile, MN-major); it
+//               also owns the TMEM allocation
+//   warp 14     MMA issuer of stage B (A = hi/lo Y in TMEM, B = P2^T in SMEM)
 //   warp 15     idle after the prologue
-// Two TMEM buffers (D_A for Y, D_B for X'') let stage A of tile i+2 run while the
-// quantizer still reads tile i.
+// TMEM holds two to four D_A slots (Y, then its hi / lo) and two or three D_B slots (X''),
+// as many as fit in 512 columns, so stage A runs ahead of the epilogue.
 // Every wait is bounded in time; on expiry the kernel records a code in the status word,
 // drains its copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -51,12 +51,12 @@ namespace {
 
 constexpr int kStages = 4;
 constexpr int kThreads = 512;  // four warpgroups
-// Register split (setmaxnreg): launched at kLaunchRegs per thread; the splitter and the
-// two quantizer warpgroups rise to kSplitRegs / kQuantRegs and the producer / MMA
-// warpgroup drops to kLowRegs. The shares add up to no more than the registers the block was
+// Register split (setmaxnreg): launched at kLaunchRegs per thread; the three epilogue
+// warpgroups rise to kEpiRegs and the producer / MMA warpgroup drops to kLowRegs. The shares add up to no more than the registers the block was
 // launched with, so setmaxnreg.inc always finds what it asks for.
-constexpr int kLaunchRegs = 128, kSplitRegs = 152, kQuantRegs = 152, kLowRegs = 56;
-static_assert(128 * (kSplitRegs + 2 * kQuantRegs + kLowRegs) <= kThreads * kLaunchRegs, "register split");
+constexpr int kEpi = 3;  // epilogue warpgroups (warps 0-11)
+constexpr int kLaunchRegs = 128, kEpiRegs = 152, kLowRegs = 56;
+static_assert(128 * (kEpi * kEpiRegs + kLowRegs) <= kThreads * kLaunchRegs, "register split");
 constexpr uint64_t kTimeoutNs = 4000000000ull;  // 4 s: far beyond any legitimate wait
 
 // status bits (device status word)
@@ -80,32 +80,41 @@ struct Geo {
   static constexpr int kOffP2 = kOffP1 + kP1Bytes;
   static constexpr int kOffX = kOffP2 + kP2Bytes;
   static constexpr int kOffOut = kOffX + kStages * kXStage;
-  static constexpr int kOffBar = kOffOut + 2 * kOutStride;
+  static constexpr int kOffBar = kOffOut + kEpi * kOutStride;
   static constexpr int kSmem = kOffBar + 4096 + 1024;       // barriers + alignment slack
-  // TMEM buffers of (D_A, D_B), 2N columns each: four when they fit (N = 64), else two.
-  static constexpr int kNbuf = (8 * N <= 512) ? 4 : 2;
-  static constexpr int kRing = 2 * kNbuf;  // row-exponent ring (see the quantizer)
+  // TMEM: kNA slots of N columns for D_A (Y, then its hi / lo) and kNB slots for D_B (X''),
+  // as many as fit in 512 columns, D_B first. Tile i uses D_A slot i % kNA and D_B slot
+  // i % kNB. Both are at most kEpi (see the MMA issuers).
+  static constexpr int kSlots = 512 / N;
+  static constexpr int kNB = kSlots / 2 < kEpi ? kSlots / 2 : kEpi;
+  static constexpr int kNA = kSlots - kNB < kEpi ? kSlots - kNB : kEpi;
+  static_assert(kNA >= 2 && kNB >= 1 && kNA <= kEpi && kNB <= kEpi, "TMEM slots");
   static constexpr int kBlocks = N / 16;          // 16-column blocks of a row
   static constexpr int kGroups = (kBlocks + 1) / 2;  // published two blocks at a time
-  static constexpr uint32_t kTmemCols = (kNbuf * 2 * N <= 256) ? 256u : 512u;
+  static constexpr uint32_t kTmemCols = ((kNA + kNB) * N <= 256) ? 256u : 512u;
 };
 
 struct Bars {
   uint64_t x_full[kStages];
   uint64_t x_empty[kStages];
-  uint64_t da_full[4];
-  uint64_t ys_full[4][4];  // per buffer: hi / lo of column group g (two 16-column blocks) written
-  uint64_t db_full[4];
-  uint64_t tm_empty[4];
-  uint64_t srow_full[8];  // row exponents of tile i published in srow[i % ring]
+  // Every barrier below is waited for by one thread or one warpgroup, phase after phase.
+  uint64_t da_full[kEpi];   // stage A of tile i done (barrier of its epilogue group i % kEpi)
+  uint64_t db_full[kEpi];   // stage B of tile i done (same)
+  uint64_t ys_full[4][4];   // D_A slot: hi / lo of column group g (two 16-column blocks) written
+  uint64_t da_free[4];      // D_A slot: stage B that read it has completed
+  uint64_t tm_empty[4];     // D_B slot: X'' read out by the epilogue
   uint64_t mma_done[2];
   uint32_t tmem_base;
   int abort;
-  int group_exit[2][2];  // per quantizer group: exit decision, one slot per use parity
-  float red[2][4];
+  int group_exit[kEpi][2];  // per epilogue group: exit decision, one slot per use parity
+  float red[kEpi][4];
   float wmax[kThreads / 32];
-  int8_t srow[8][128];  // per-row power-of-two exponent of Y, ring of 2 * buffers tiles
 };
+static_assert(sizeof(Bars) <= 4096, "barrier block");
+template <int N>
+constexpr bool smem_fits() { return Geo<N>::kSmem <= 232448; }  // 227 KB opt-in per block
+static_assert(smem_fits<64>() && smem_fits<80>() && smem_fits<96>() && smem_fits<112>() && smem_fits<128>(),
+              "shared memory");
 
 // ------------------------------------------------------------------------------------
 // PTX wrappers
@@ -126,6 +135,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t b, uint32_t parity) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(b), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// non-blocking test of a phase (the event loop of the MMA issuer must not be suspended)
+__device__ __forceinline__ bool mbar_test(uint32_t b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(b), "r"(parity)
@@ -227,6 +248,38 @@ __device__ __forceinline__ void mma_ts_lo(uint32_t d, uint32_t a_tmem, uint32_t 
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %3, p;\n\t}" ::"r"(d),
       "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(acc), "n"(kDescHi)
       : "memory");
+}
+
+// Warp-wide forms for the issuing warp: every lane runs the same code (so descriptors stay
+// warp-uniform) and one elected lane issues the instruction.
+__device__ __forceinline__ void mma_ss_e(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_e(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit_e(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ uint64_t desc64(uint32_t saddr, uint32_t lbo) {
+  return (uint64_t(kDescHi) << 32) | desc_lo(saddr, lbo);
 }
 
 // Instruction descriptor, kind::f16, fp32 accumulate, M = 128.
@@ -409,18 +462,19 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       mbar_init(&bars->x_full[s], 1);
       mbar_init(&bars->x_empty[s], 1);
     }
-    for (int b = 0; b < 4; ++b) {
-      mbar_init(&bars->da_full[b], 1);
-      for (int g = 0; g < 4; ++g) mbar_init(&bars->ys_full[b][g], 4);
-      mbar_init(&bars->db_full[b], 1);
-      mbar_init(&bars->tm_empty[b], 4);
+    for (int a = 0; a < 4; ++a) {
+      for (int g = 0; g < 4; ++g) mbar_init(&bars->ys_full[a][g], 4);
+      mbar_init(&bars->da_free[a], 1);
+      mbar_init(&bars->tm_empty[a], 4);
     }
-    for (int r = 0; r < 8; ++r) mbar_init(&bars->srow_full[r], 4);
+    for (int g = 0; g < kEpi; ++g) {
+      mbar_init(&bars->da_full[g], 1);
+      mbar_init(&bars->db_full[g], 1);
+    }
     mbar_init(&bars->mma_done[0], 1);
     mbar_init(&bars->mma_done[1], 1);
     bars->abort = 0;
-    bars->group_exit[0][0] = bars->group_exit[0][1] = 0;
-    bars->group_exit[1][0] = bars->group_exit[1][1] = 0;
+    for (int g = 0; g < kEpi; ++g) bars->group_exit[g][0] = bars->group_exit[g][1] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -504,90 +558,118 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     }
   } else if (warp == 13 || warp == 14) {
     // ---------------- MMA issuers ----------------
-    // Warp 13 issues the MMAs of the even local tiles, warp 14 those of the odd tiles, so a
-    // slow tile on one side does not hold up the other; the tensor pipe interleaves the
-    // two streams. Tile i uses TMEM buffer i % NB. A(i) may overwrite D_A once B(i-NB) has
-    // read its hi / lo Y; B(i) may overwrite D_B once the quantizer has read the X'' of
-    // tile i-NB. With four buffers each issuer runs stage A one of its tiles ahead.
+    // Warp 13 issues stage A of every tile, warp 14 stage B, each in tile order and each
+    // with blocking waits (a waiting warp takes no issue slots from the epilogue warps on
+    // its sub-partition). The whole warp runs the loop, so descriptors stay warp-uniform,
+    // and one elected lane issues.
+    //   stage A of tile a: x tile landed; D_A slot free (stage B of tile a - kNA done).
+    //   stage B of tile b: D_B slot free (tile b - kNB read out); then each pair of
+    //                      16-column blocks of hi / lo as soon as it is published.
+    // Every barrier has one waiter that takes its phases in order. A waiter is never two
+    // phases behind: stage A of tile i + kEpi waits for stage B of tile i + kEpi - kNA,
+    // issued after stage B of tile i (kNA <= kEpi), which waits for the split of tile i;
+    // stage B of tile i + kEpi is issued after stage B of tile i + kNB (kNB <= kEpi), which
+    // waits for the epilogue to read tile i out.
     setmaxnreg_dec<kLowRegs>();
+    const int n_local = (blockIdx.x < num_tiles) ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     const int mb = warp - 13;
-    if (lane == 0) {
-      const int n_local = (blockIdx.x < num_tiles) ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    if (mb == 0) {
       constexpr uint32_t kIdA = idesc_f16(!kF16, !kF16, true, N);
-      constexpr uint32_t kIdB = idesc_f16(false, false, false, N);
-      auto issue_a = [&](int i) -> bool {
-        const int s = i % kStages, b = i % G::kNbuf, u = i / G::kNbuf;
-        if (!wait_bounded(&bars->x_full[s], (i / kStages) & 1, bars, p.status, kStMmaXFull)) return false;
-        if (u >= 1 && !wait_bounded(&bars->db_full[b], (u - 1) & 1, bars, p.status, kStMmaTmemEmpty))
-          return false;
+      const uint64_t p1_desc = desc64(sbase + G::kOffP1, 16);
+      for (int a = 0; a < n_local; ++a) {
+        const int s = a % kStages, sa = a % G::kNA;
+        if (!warp_wait(&bars->x_full[s], (a / kStages) & 1, bars, p.status, kStMmaXFull)) break;
+        if (a >= G::kNA && !warp_wait(&bars->da_free[sa], ((a / G::kNA) - 1) & 1, bars, p.status, kStMmaTmemEmpty))
+          break;
         tc_fence_after();
-        const uint32_t d = tmem + uint32_t(b * 2 * N);
-        // low descriptor words: base + a compile-time offset per MMA (about five
-        // instructions per MMA, so the issue keeps up with the tensor pipe)
-        const uint32_t a_lo = desc_lo(sbase + G::kOffP1, 16);
-        const uint32_t x_lo = desc_lo(sbase + G::kOffX + s * G::kXStage, 16384);
+        const uint32_t d = tmem + uint32_t(sa * N);
+        const uint64_t x_desc = desc64(sbase + G::kOffX + s * G::kXStage, 16384);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss_lo(d, a_lo + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), x_lo + ((kk * 2048) >> 4), kIdA,
-                    kk > 0 ? 1u : 0u);
-        mma_commit(&bars->x_empty[s]);
-        mma_commit(&bars->da_full[b]);
-        return true;
-      };
-      auto issue_b = [&](int i) -> bool {
-        const int b = i % G::kNbuf, u = i / G::kNbuf;
-        if (!wait_bounded(&bars->tm_empty[b], (u & 1) ^ 1, bars, p.status, kStMmaTmemEmpty)) return false;
-        const uint32_t d = tmem + uint32_t(b * 2 * N + N);
-        const uint32_t a0 = tmem + uint32_t(b * 2 * N);
-        const uint32_t p2_lo = desc_lo(sbase + G::kOffP2, 16);
-        // K-steps are issued as the splitter publishes each pair of 16-column blocks, so
-        // stage B runs alongside the split instead of after it
+          mma_ss_e(d, p1_desc + uint64_t(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                   x_desc + uint64_t((kk * 2048) >> 4), kIdA, kk > 0 ? 1u : 0u);
+        mma_commit_e(&bars->x_empty[s]);
+        mma_commit_e(&bars->da_full[a % kEpi]);
+      }
+    } else {
+      constexpr uint32_t kIdB = idesc_f16(false, false, false, N);
+      const uint64_t p2_desc = desc64(sbase + G::kOffP2, 16);
+      bool ok = true;
+      for (int b = 0; ok && b < n_local; ++b) {
+        const int sa = b % G::kNA;
+        if (b >= G::kNB &&
+            !warp_wait(&bars->tm_empty[b % G::kNB], ((b / G::kNB) - 1) & 1, bars, p.status, kStMmaTmemEmpty))
+          break;
+        const uint32_t d = tmem + uint32_t((G::kNA + b % G::kNB) * N);
+        const uint32_t a0 = tmem + uint32_t(sa * N);
 #pragma unroll
         for (int g = 0; g < G::kGroups; ++g) {
-          if (!wait_bounded(&bars->ys_full[b][g], u & 1, bars, p.status, kStMmaYsFull)) return false;
+          ok = warp_wait(&bars->ys_full[sa][g], (b / G::kNA) & 1, bars, p.status, kStMmaYsFull);
+          if (!ok) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 2 * g; kk < 2 * g + 2 && kk < G::kBlocks; ++kk) {
 #pragma unroll
             for (int h = 0; h < 2; ++h)
-              mma_ts_lo(d, a0 + uint32_t(kk * 16 + h * 8), p2_lo + (((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4),
-                        kIdB, (h | kk) != 0 ? 1u : 0u);
+              mma_ts_e(d, a0 + uint32_t(kk * 16 + h * 8),
+                       p2_desc + uint64_t(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4), kIdB,
+                       (h | kk) != 0 ? 1u : 0u);
           }
         }
-        mma_commit(&bars->db_full[b]);
-        return true;
-      };
-      constexpr int kAhead = G::kNbuf / 2 - 1;  // stage-A lookahead, in this issuer's tiles
-      bool ok = true;
-      for (int k = 0; ok && k < kAhead; ++k)
-        if (mb + 2 * k < n_local) ok = issue_a(mb + 2 * k);
-      for (int i = mb; ok && i < n_local; i += 2) {
-        if (i + 2 * kAhead < n_local) ok = issue_a(i + 2 * kAhead);
-        if (ok) ok = issue_b(i);
+        if (!ok) break;
+        mma_commit_e(&bars->db_full[b % kEpi]);
+        mma_commit_e(&bars->da_free[sa]);
       }
-      // every MMA issued by this thread has completed before TMEM is released
-      mma_commit(&bars->mma_done[mb]);
-      const uint32_t b = smem_u32(&bars->mma_done[mb]);
+    }
+    // every MMA issued by this warp has completed before TMEM is released
+    mma_commit_e(&bars->mma_done[mb]);
+    if (lane == 0) {
+      const uint32_t bd = smem_u32(&bars->mma_done[mb]);
       const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(b, 0)) {
+      while (!mbar_try_wait(bd, 0)) {
         if (globaltimer() - t0 > kTimeoutNs) { atomicOr(p.status, kStMmaDone); break; }
       }
     }
     __syncwarp();
   } else if (warp == 15) {
     setmaxnreg_dec<kLowRegs>();  // idle warp of the producer / MMA warpgroup
-  } else if (warp < 4) {
-    // ---------------- splitter: Y -> per-row power-of-two scale -> fp16 hi / lo ----------------
-    setmaxnreg_inc<kSplitRegs>();
-    const int q = warp & 3;
+  } else {
+    // ---------------- epilogue warpgroups: split, then quantize, the same tile ----------------
+    // Group eg takes the local tiles i = eg (mod kEpi). For its tile it first splits Y
+    // (D_A) into fp16 hi / lo for stage B, publishing each pair of 16-column blocks as
+    // soon as it is in TMEM, then waits for stage B and turns X'' (D_B) into codes and
+    // scales. A thread owns one row (TMEM lane) throughout, so its row exponent stays in
+    // a register. The groups work on consecutive tiles at the same time, so the split of
+    // one tile overlaps the split and the encoding of the next ones.
+    setmaxnreg_inc<kEpiRegs>();
+    const int eg = warp >> 2;              // group: tile residue and staging buffer
+    const int q = warp & 3;                // TMEM lane quarter of this warp
     const int row = q * 32 + lane;
     const uint32_t t_lane = tmem + (uint32_t(q * 32) << 16);
-    int i = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
-      const int b = i % G::kNbuf, u = i / G::kNbuf;
-      const uint32_t colA = uint32_t(b * 2 * N);
+    const bool leader = (q == 0) && lane == 0;
+    const int bar_id = 1 + eg;
+    const int tok_in_tile = row / M;
+    const int m_row = row % M;
+    uint8_t* s_out = smem + G::kOffOut + eg * G::kOutStride;
+    const uint32_t s_out_u32 = sbase + G::kOffOut + eg * G::kOutStride;
+    constexpr int NS = N / 16;                 // 16-column segments
+
+    int jj = 0;  // tiles done by this group
+    for (int i = eg, tile = blockIdx.x + eg * gridDim.x; tile < num_tiles;
+         i += kEpi, tile += kEpi * gridDim.x, ++jj) {
+      const int64_t grow = int64_t(tile) * 128 + row;
+      const int64_t rows_left = rows_total - int64_t(tile) * 128;
+      const int valid_rows = rows_left < 128 ? int(rows_left) : 128;
+      const bool row_valid = grow < rows_total;
+      const int sa = i % G::kNA, sb = i % G::kNB;
+
+      // ---- split: Y -> per-row power-of-two scale -> fp16 hi / lo in place ----
+      const uint32_t colA = uint32_t(sa * N);
       int s_exp = 0;
-      const bool ok = warp_wait(&bars->da_full[b], u & 1, bars, p.status, kStEpiAFull);
+      // tile i is phase jj of this group's stage-A barrier; the group waited for the
+      // previous phase itself, and the next one (tile i + kEpi) cannot complete before this
+      // split is published (see the MMA issuers)
+      bool ok = warp_wait(&bars->da_full[eg], jj & 1, bars, p.status, kStEpiAFull);
       if (ok) {
         tc_fence_after();
         // one TMEM round trip: the whole row, then the row maximum as a shallow tree
@@ -598,7 +680,6 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
         s_exp = prescale_exp(absmax<N>(y));
         const float sc = exp2i(s_exp);
         const float2 sc2 = make_float2(sc, sc);
-        bars->srow[i % G::kRing][row] = int8_t(s_exp);
         // each 16-column block of the row becomes 8 words of hi then 8 words of lo; every
         // pair of blocks is published on its own barrier as soon as it is in TMEM
 #pragma unroll
@@ -618,60 +699,31 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->ys_full[b][g]);
+          if (lane == 0) mbar_arrive(&bars->ys_full[sa][g]);
         }
       } else {
         // a failed wait still publishes every group, so the MMA issuer is not left waiting
         tc_fence_before();
         __syncwarp();
         if (lane == 0)
-          for (int g = 0; g < G::kGroups; ++g) mbar_arrive(&bars->ys_full[b][g]);
+          for (int g = 0; g < G::kGroups; ++g) mbar_arrive(&bars->ys_full[sa][g]);
       }
-      if (lane == 0) mbar_arrive(&bars->srow_full[i % G::kRing]);
-      if (!ok) break;
-    }
-  } else {
-    // ---------------- quantizers: X'' = D * 2^crow -> codes and scales ----------------
-    // Two warpgroups, for the even and the odd local tiles. A thread reads its whole
-    // row of X'' in one TMEM round trip and releases the buffer at once, so stage B of tile
-    // i+2 can start while tile i is still being encoded.
-    setmaxnreg_inc<kQuantRegs>();
-    const int qb = (warp >> 2) - 1;        // tile parity and staging buffer of this group
-    const int q = warp & 3;
-    const int row = q * 32 + lane;
-    const uint32_t t_lane = tmem + (uint32_t(q * 32) << 16);
-    const bool leader = (q == 0) && lane == 0;
-    const int bar_id = 1 + qb;
-    const int tok_in_tile = row / M;
-    const int m_row = row % M;
-    uint8_t* s_out = smem + G::kOffOut + qb * G::kOutStride;
-    const uint32_t s_out_u32 = sbase + G::kOffOut + qb * G::kOutStride;
-    constexpr int NS = N / 16;                 // 16-column segments
 
-    int jj = 0;  // use count of this buffer
-    for (int i = qb, tile = blockIdx.x + qb * gridDim.x; tile < num_tiles;
-         i += 2, tile += 2 * gridDim.x, ++jj) {
-      const int64_t grow = int64_t(tile) * 128 + row;
-      const int64_t rows_left = rows_total - int64_t(tile) * 128;
-      const int valid_rows = rows_left < 128 ? int(rows_left) : 128;
-      const bool row_valid = grow < rows_total;
-
-      const int b = i % G::kNbuf, u = i / G::kNbuf;
-      const uint32_t colB = uint32_t(b * 2 * N + N);
-      bool ok = warp_wait(&bars->db_full[b], u & 1, bars, p.status, kStEpiBFull);
-      // the splitter's row exponents of this tile, in slot i % ring (ring = 2 NB). The
-      // splitter reaches tile i + ring only after this group has released D_B of tile i
-      // (A(i+ring) needs B(i+NB), which needs that release), so this wait is never more
-      // than one phase of srow_full[i % ring] behind, and the slot is not overwritten
-      // before it is read.
-      ok = ok && warp_wait(&bars->srow_full[i % G::kRing], (i / G::kRing) & 1, bars, p.status, kStEpiAFull);
+      // keeps the compiler from moving work of one phase into the other, which would
+      // hold both rows in registers at once
+      asm volatile("" ::: "memory");
+      // ---- quantize: X'' = D * 2^crow -> codes and scales ----
+      // D_B of tile i is free again for stage B of tile i + NB as soon as this group has
+      // read it, so the whole row comes out of TMEM in one round trip first.
+      // phase jj of this group's stage-B barrier; stage B of tile i + kEpi cannot complete
+      // before this group has read D_B out (see the MMA issuers)
+      const uint32_t colB = uint32_t((G::kNA + sb) * N);
+      ok = ok && warp_wait(&bars->db_full[eg], jj & 1, bars, p.status, kStEpiBFull);
       float d[N];
-      int s_exp = 0;
       if (ok) {
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < NS; ++c) tmem_ld16(t_lane + colB + c * 16, d + c * 16);
-        s_exp = bars->srow[i % G::kRing][row];
         tmem_wait_ld();
       } else {
 #pragma unroll
@@ -679,7 +731,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->tm_empty[b]);
+      if (lane == 0) mbar_arrive(&bars->tm_empty[sb]);
       const int crow = -(s_exp + t_exp);
       const float fcrow = exp2i(crow);
 
@@ -690,9 +742,9 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
           for (int e = 0; e < N; e += 4)
             dst[e / 4] = make_float4(d[e] * fcrow, d[e + 1] * fcrow, d[e + 2] * fcrow, d[e + 3] * fcrow);
         }
-        if (leader) bars->group_exit[qb][jj & 1] = *reinterpret_cast<volatile int*>(&bars->abort) | int(!ok);
+        if (leader) bars->group_exit[eg][jj & 1] = *reinterpret_cast<volatile int*>(&bars->abort) | int(!ok);
         named_bar(bar_id, 128);
-        if (bars->group_exit[qb][jj & 1]) break;
+        if (bars->group_exit[eg][jj & 1]) break;
         continue;
       } else {
         float smax[NS];
@@ -705,11 +757,11 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
 #pragma unroll
           for (int sg = 0; sg < NS; ++sg) rmax = fmaxf(rmax, smax[sg]);
           const float wm = warp_max(rmax * fcrow);
-          if (lane == 0) bars->red[qb][q] = wm;
+          if (lane == 0) bars->red[eg][q] = wm;
           named_bar(bar_id, 128);
           float amax = 0.0f;
           const int q0 = (tok_in_tile * M) >> 5, nq = (M + 31) >> 5;
-          for (int qq = 0; qq < nq; ++qq) amax = fmaxf(amax, bars->red[qb][q0 + qq]);
+          for (int qq = 0; qq < nq; ++qq) amax = fmaxf(amax, bars->red[eg][q0 + qq]);
           const float qs = per_token_scale(amax, p.clip_ratio);
           const float inv = qs > 0.0f ? __frcp_rn(qs) : 0.0f;
           if (row_valid && m_row == 0) p.quant_scale[grow / M] = qs;
@@ -787,7 +839,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
           *reinterpret_cast<uint2*>(s_out + row * (N / 2) + sg * 8) = make_uint2(words[0], words[1]);
         }
         fence_proxy_async();
-        if (leader) bars->group_exit[qb][jj & 1] = *reinterpret_cast<volatile int*>(&bars->abort) | int(!ok);
+        if (leader) bars->group_exit[eg][jj & 1] = *reinterpret_cast<volatile int*>(&bars->abort) | int(!ok);
         named_bar(bar_id, 128);
         if (leader) {
           const int64_t row0 = int64_t(tile) * 128;
@@ -796,7 +848,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
             bulk_store(p.scales + (row0 * N) / 32, s_out_u32 + G::kCodeBytes, uint32_t((valid_rows * N) / 32));
           bulk_commit();
         }
-        if (bars->group_exit[qb][jj & 1]) break;
+        if (bars->group_exit[eg][jj & 1]) break;
       }
     }
     if (leader) bulk_wait_all();
