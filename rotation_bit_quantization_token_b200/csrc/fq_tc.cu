@@ -672,34 +672,52 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       bool ok = warp_wait(&bars->da_full[eg], jj & 1, bars, p.status, kStEpiAFull);
       if (ok) {
         tc_fence_after();
-        // one TMEM round trip: the whole row, then the row maximum as a shallow tree
+        // the row comes out of TMEM in two batches; the maximum of the first is formed
+        // while the second is in flight
+        constexpr int kB1 = (G::kBlocks + 1) / 2;
         float y[N];
 #pragma unroll
-        for (int c = 0; c < N / 16; ++c) tmem_ld16(t_lane + colA + c * 16, y + c * 16);
+        for (int c = 0; c < kB1; ++c) tmem_ld16(t_lane + colA + c * 16, y + c * 16);
         tmem_wait_ld();
-        s_exp = prescale_exp(absmax<N>(y));
+#pragma unroll
+        for (int c = kB1; c < G::kBlocks; ++c) tmem_ld16(t_lane + colA + c * 16, y + c * 16);
+        const float m1 = absmax<kB1 * 16>(y);
+        tmem_wait_ld();
+        s_exp = prescale_exp(fmaxf(m1, absmax<N - kB1 * 16>(y + kB1 * 16)));
         const float sc = exp2i(s_exp);
         const float2 sc2 = make_float2(sc, sc);
         // each 16-column block of the row becomes 8 words of hi then 8 words of lo; every
-        // pair of blocks is published on its own barrier as soon as it is in TMEM
+        // pair of blocks is published on its own barrier as soon as its stores have
+        // landed, and the next pair is converted while they are in flight
+        auto convert = [&](int c, uint32_t* hl) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float2 v = __fmul2_rn(make_float2(y[c * 16 + 2 * e], y[c * 16 + 2 * e + 1]), sc2);
+            const __half2 h = __float22half2_rn(v);
+            hl[e] = h2_bits(h);
+            hl[8 + e] = h2_bits(__float22half2_rn(residual2(h, v)));
+          }
+        };
+        uint32_t hl[2][2][16];  // [pair parity][block of the pair][words]
+        convert(0, hl[0][0]);
+        if (G::kBlocks > 1) convert(1, hl[0][1]);
+        tmem_st16(t_lane + colA, hl[0][0]);
+        if (G::kBlocks > 1) tmem_st16(t_lane + colA + 16, hl[0][1]);
 #pragma unroll
         for (int g = 0; g < G::kGroups; ++g) {
-#pragma unroll
-          for (int c = 2 * g; c < 2 * g + 2 && c < G::kBlocks; ++c) {
-            uint32_t hl[16];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float2 v = __fmul2_rn(make_float2(y[c * 16 + 2 * e], y[c * 16 + 2 * e + 1]), sc2);
-              const __half2 h = __float22half2_rn(v);
-              hl[e] = h2_bits(h);
-              hl[8 + e] = h2_bits(__float22half2_rn(residual2(h, v)));
-            }
-            tmem_st16(t_lane + colA + c * 16, hl);
+          const int nx = (g + 1) & 1;
+          if (g + 1 < G::kGroups) {
+            convert(2 * g + 2, hl[nx][0]);
+            if (2 * g + 3 < G::kBlocks) convert(2 * g + 3, hl[nx][1]);
           }
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars->ys_full[sa][g]);
+          if (g + 1 < G::kGroups) {
+            tmem_st16(t_lane + colA + (2 * g + 2) * 16, hl[nx][0]);
+            if (2 * g + 3 < G::kBlocks) tmem_st16(t_lane + colA + (2 * g + 3) * 16, hl[nx][1]);
+          }
         }
       } else {
         // a failed wait still publishes every group, so the MMA issuer is not left waiting
