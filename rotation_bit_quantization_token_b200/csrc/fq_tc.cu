@@ -130,14 +130,18 @@ __device__ __forceinline__ uint64_t globaltimer() {
 __device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
 }
+// Waits for a phase to complete, with the thread suspended in hardware until it does or
+// kSuspendNs pass (a short hint would make waiting warps spin, taking issue slots from the
+// warps that work on their sub-partition).
+constexpr uint32_t kSuspendNs = 1000000;
 __device__ __forceinline__ bool mbar_try_wait(uint32_t b, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(b), "r"(parity)
+      : "r"(b), "r"(parity), "n"(kSuspendNs)
       : "memory");
   return ok != 0;
 }
@@ -380,21 +384,21 @@ __device__ __forceinline__ float2 residual2(__half2 h, float2 v) {
       : "r"(hb), "f"(v.x), "f"(v.y));
   return r;
 }
-// Bounded wait on an mbarrier phase. On expiry sets the abort flag and a status bit.
+// Bounded wait on an mbarrier phase. On expiry sets the abort flag and a status bit. Each
+// unsuccessful try lasts up to kSuspendNs, so the abort flag and the clock are checked
+// after every one.
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, Bars* bars, uint32_t* status,
                                           uint32_t code) {
   const uint32_t b = smem_u32(bar);
   if (mbar_try_wait(b, parity)) return true;
   const uint64_t t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
+  for (;;) {
     if (mbar_try_wait(b, parity)) return true;
-    if ((it & 63u) == 0u) {
-      if (*reinterpret_cast<volatile int*>(&bars->abort)) return false;
-      if (globaltimer() - t0 > kTimeoutNs) {
-        *reinterpret_cast<volatile int*>(&bars->abort) = 1;
-        atomicOr(status, code);
-        return false;
-      }
+    if (*reinterpret_cast<volatile int*>(&bars->abort)) return false;
+    if (globaltimer() - t0 > kTimeoutNs) {
+      *reinterpret_cast<volatile int*>(&bars->abort) = 1;
+      atomicOr(status, code);
+      return false;
     }
   }
 }
