@@ -71,7 +71,12 @@ struct Geo {
   static_assert(N % 16 == 0 && N >= 64 && N <= 128, "tensor-core kernel covers N in [64,128], N % 16 == 0");
   static constexpr int kAtoms = (N + 63) / 64;              // 64-element swizzle atoms along N
   static constexpr int kXStage = kAtoms * 128 * 128;        // bytes per x stage
-  static constexpr int kP1Bytes = 2 * 128 * 128;            // BD(P1): 128 x 128, two K atoms
+  // BD(P1) sits in TMEM (64 columns; stage A is then a TS MMA that reads only the x tile
+  // from shared memory, 3.5 KB instead of 7.5 KB per MMA at N = 112) when four N-column
+  // slots still fit beside it; otherwise in shared memory, 128 x 128, two K atoms (SS).
+  static constexpr bool kP1Tmem = (512 - 64) / N >= 4;
+  static constexpr uint32_t kP1Col = 448;                   // its first TMEM column
+  static constexpr int kP1Bytes = kP1Tmem ? 0 : 2 * 128 * 128;
   static constexpr int kP2Bytes = kAtoms * N * 128;         // P2^T: N rows, kAtoms K atoms
   static constexpr int kCodeBytes = 128 * N / 2;
   static constexpr int kScaleBytes = 4 * N;                 // 128 rows x N/32 groups
@@ -85,13 +90,13 @@ struct Geo {
   // TMEM: kNA slots of N columns for D_A (Y, then its hi / lo) and kNB slots for D_B (X''),
   // as many as fit in 512 columns, D_B first. Tile i uses D_A slot i % kNA and D_B slot
   // i % kNB. Both are at most kEpi (see the MMA issuers).
-  static constexpr int kSlots = 512 / N;
+  static constexpr int kSlots = (kP1Tmem ? 448 : 512) / N;
   static constexpr int kNB = kSlots / 2 < kEpi ? kSlots / 2 : kEpi;
   static constexpr int kNA = kSlots - kNB < kEpi ? kSlots - kNB : kEpi;
   static_assert(kNA >= 2 && kNB >= 1 && kNA <= kEpi && kNB <= kEpi, "TMEM slots");
   static constexpr int kBlocks = N / 16;          // 16-column blocks of a row
   static constexpr int kGroups = (kBlocks + 1) / 2;  // published two blocks at a time
-  static constexpr uint32_t kTmemCols = ((kNA + kNB) * N <= 256) ? 256u : 512u;
+  static constexpr uint32_t kTmemCols = (!kP1Tmem && (kNA + kNB) * N <= 256) ? 256u : 512u;
 };
 
 struct Bars {
@@ -145,18 +150,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t b, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// non-blocking test of a phase (the event loop of the MMA issuer must not be suspended)
-__device__ __forceinline__ bool mbar_test(uint32_t b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(b), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
 __device__ __forceinline__ void mbar_arrive(uint64_t* b) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
 }
@@ -200,11 +193,6 @@ __device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
   uint32_t r[16];
   asm volatile(
@@ -234,26 +222,6 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 // leading byte offset (>> 4); shared-memory addresses are below 2^18, so no masking.
 constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
 __device__ __forceinline__ uint32_t desc_lo(uint32_t saddr, uint32_t lbo) { return (saddr >> 4) | ((lbo >> 4) << 16); }
-__device__ __forceinline__ void mma_ss_lo(uint32_t d, uint32_t a_lo, uint32_t b_lo, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "mov.b64 da, {%1, %5};\n\t"
-      "mov.b64 db, {%2, %5};\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n\t}" ::"r"(d),
-      "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(acc), "n"(kDescHi)
-      : "memory");
-}
-__device__ __forceinline__ void mma_ts_lo(uint32_t d, uint32_t a_tmem, uint32_t b_lo, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "mov.b64 db, {%2, %5};\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %3, p;\n\t}" ::"r"(d),
-      "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(acc), "n"(kDescHi)
-      : "memory");
-}
-
 // Warp-wide forms for the issuing warp: every lane runs the same code (so descriptors stay
 // warp-uniform) and one elected lane issues the instruction.
 __device__ __forceinline__ void mma_ss_e(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
@@ -490,7 +458,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
 
   // BD(P1): 128 x 128, K-major, 128B swizzle; element (r, k) = P1[r % M][k % M] on the
   // diagonal blocks (r / M == k / M), else 0.
-  for (int c = tid; c < 128 * 16; c += kThreads) {
+  for (int c = tid; !G::kP1Tmem && c < 128 * 16; c += kThreads) {
     const int r = c >> 4, kc = c & 15, k = kc * 8;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (r / M == k / M)
@@ -531,6 +499,32 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+  if constexpr (G::kP1Tmem) {
+    // BD(P1) into TMEM as the A operand of stage A: lane r holds row r, column c the
+    // elements (r, 2c) and (r, 2c + 1) in its low and high halves
+    if (tid < 128) {
+      const int r = tid;
+      uint32_t w[64];
+#pragma unroll
+      for (int kc = 0; kc < 16; ++kc) {
+        const int k = kc * 8;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (r / M == k / M)
+          v = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.P1) + (r % M) * M + (k % M));
+        w[4 * kc] = v.x;
+        w[4 * kc + 1] = v.y;
+        w[4 * kc + 2] = v.z;
+        w[4 * kc + 3] = v.w;
+      }
+      const uint32_t t_row = tmem + (uint32_t(warp * 32) << 16) + G::kP1Col;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) tmem_st16(t_row + 16 * j, w + 16 * j);
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
 
   if (warp == 12) {
     // ---------------- TMA producer ----------------
@@ -589,9 +583,14 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
         const uint32_t d = tmem + uint32_t(sa * N);
         const uint64_t x_desc = desc64(sbase + G::kOffX + s * G::kXStage, 16384);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss_e(d, p1_desc + uint64_t(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
-                   x_desc + uint64_t((kk * 2048) >> 4), kIdA, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk) {
+          if constexpr (G::kP1Tmem)
+            mma_ts_e(d, tmem + G::kP1Col + uint32_t(kk * 8), x_desc + uint64_t((kk * 2048) >> 4), kIdA,
+                     kk > 0 ? 1u : 0u);
+          else
+            mma_ss_e(d, p1_desc + uint64_t(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                     x_desc + uint64_t((kk * 2048) >> 4), kIdA, kk > 0 ? 1u : 0u);
+        }
         mma_commit_e(&bars->x_empty[s]);
         mma_commit_e(&bars->da_full[a % kEpi]);
       }
