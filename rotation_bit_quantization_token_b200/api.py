@@ -64,6 +64,7 @@ class FlatQuant:
         code = {"auto": _lib.FQ_KERNEL_AUTO, "general": _lib.FQ_KERNEL_GENERAL,
                 "tcgen05": _lib.FQ_KERNEL_TCGEN05}[kernel]
         _lib.check(self._lib.fq_set_kernel(self._h, code), "fq_set_kernel")
+        self.kernel = kernel
 
     @property
     def last_kernel(self):
@@ -181,11 +182,15 @@ def debug_rotate(x, P1, P2, kernel="auto"):
 
 
 class HostPipeline:
-    """End-to-end use from host memory: pinned host inputs are copied to device staging
-    buffers, the operator runs, and the packed outputs and scales are copied back, all on
-    one stream. The device buffers are allocated once, in the constructor."""
+    """End-to-end use from host memory. The tokens are processed in `chunks` equal slices:
+    the host-to-device copy of slice c + 1, the operator on slice c and the device-to-host
+    copy of slice c - 1 run on three streams at once (the copy engines work in both
+    directions together), so a step costs about its larger transfer instead of the sum.
+    Device buffers, streams and the per-slice handle are allocated once, in the
+    constructor. With chunks = 1, or when K is not a multiple of `chunks`, everything runs
+    on the caller's stream in one slice."""
 
-    def __init__(self, fq: FlatQuant, mode, out_dtype="int4", device=None):
+    def __init__(self, fq: FlatQuant, mode, out_dtype="int4", device=None, chunks=8):
         self.fq = fq
         self.mode = mode
         self.out_dtype = out_dtype
@@ -203,6 +208,12 @@ class HostPipeline:
         else:
             self.out = torch.empty((K, M * N // 2), dtype=torch.uint8, device=dev)
             self.scale = torch.empty((K, -(-M * N // 64), 2), dtype=torch.uint8, device=dev)
+        self.chunks = chunks if chunks >= 1 and K % chunks == 0 else 1
+        self.kc = K // self.chunks
+        if self.chunks > 1:
+            self.fq_c = FlatQuant(self.kc, M, N, fq.dtype, kernel=getattr(fq, "kernel", "auto"))
+            self.s_in = torch.cuda.Stream(dev)
+            self.s_out = torch.cuda.Stream(dev)
 
     def host_outputs(self):
         """Pinned host buffers shaped like the outputs."""
@@ -215,19 +226,51 @@ class HostPipeline:
     def d2h_bytes(self):
         return sum(t.numel() * t.element_size() for t in (self.out, self.scale))
 
+    def _launch(self, fq, x, out, scale, clip_ratio, dst_type_max, s):
+        if self.mode == "per_token":
+            fq.quantize_per_token(x, self.P1, self.P2, clip_ratio, self.out_dtype,
+                                  out=out, quant_scale=scale, stream=s)
+        else:
+            fq.quantize_mx(x, self.P1, self.P2, dst_type_max, out=out, scales=scale, stream=s)
+
     def run(self, x_host, P1_host, P2_host, out_host, scale_host, clip_ratio=1.0,
             dst_type_max=0.0, stream=None):
         s = stream if stream is not None else torch.cuda.current_stream()
-        with torch.cuda.stream(s):
-            self.x.copy_(x_host, non_blocking=True)
+        if self.chunks == 1:
+            with torch.cuda.stream(s):
+                self.x.copy_(x_host, non_blocking=True)
+                self.P1.copy_(P1_host, non_blocking=True)
+                self.P2.copy_(P2_host, non_blocking=True)
+                self._launch(self.fq, self.x, self.out, self.scale, clip_ratio, dst_type_max, s)
+                out_host.copy_(self.out, non_blocking=True)
+                scale_host.copy_(self.scale, non_blocking=True)
+            return out_host, scale_host
+        # the side streams start after everything queued on the caller's stream so far
+        # (the previous step included), and the caller's stream ends after the last copy out
+        start = torch.cuda.Event()
+        start.record(s)
+        self.s_in.wait_event(start)
+        self.s_out.wait_event(start)
+        with torch.cuda.stream(self.s_in):
             self.P1.copy_(P1_host, non_blocking=True)
             self.P2.copy_(P2_host, non_blocking=True)
-            if self.mode == "per_token":
-                self.fq.quantize_per_token(self.x, self.P1, self.P2, clip_ratio, self.out_dtype,
-                                           out=self.out, quant_scale=self.scale, stream=s)
-            else:
-                self.fq.quantize_mx(self.x, self.P1, self.P2, dst_type_max, out=self.out,
-                                    scales=self.scale, stream=s)
-            out_host.copy_(self.out, non_blocking=True)
-            scale_host.copy_(self.scale, non_blocking=True)
+        for c in range(self.chunks):
+            sl = slice(c * self.kc, (c + 1) * self.kc)
+            with torch.cuda.stream(self.s_in):
+                self.x[sl].copy_(x_host[sl], non_blocking=True)
+                landed = torch.cuda.Event()
+                landed.record(self.s_in)
+            s.wait_event(landed)
+            with torch.cuda.stream(s):
+                self._launch(self.fq_c, self.x[sl], self.out[sl], self.scale[sl], clip_ratio,
+                             dst_type_max, s)
+                done = torch.cuda.Event()
+                done.record(s)
+            self.s_out.wait_event(done)
+            with torch.cuda.stream(self.s_out):
+                out_host[sl].copy_(self.out[sl], non_blocking=True)
+                scale_host[sl].copy_(self.scale[sl], non_blocking=True)
+        end = torch.cuda.Event()
+        end.record(self.s_out)
+        s.wait_event(end)
         return out_host, scale_host

@@ -14,7 +14,7 @@ import torch
 
 import oracle
 from parity_util import compare_mx, compare_per_token, rotate_close, unpack_nibbles
-from rotation_bit_quantization_token_b200 import FlatQuant, FQError, _lib
+from rotation_bit_quantization_token_b200 import FlatQuant, FQError, HostPipeline, _lib
 from rotation_bit_quantization_token_b200.workloads import WORKLOADS, make_inputs
 
 pytestmark = pytest.mark.gpu
@@ -182,6 +182,30 @@ def test_deterministic_and_int32_same_bytes():
         m1 = fq.quantize_mx(x, P1, P2, 10.0)
         m2 = fq.quantize_mx(x, P1, P2, 10.0)
         assert torch.equal(m1[0], m2[0]) and torch.equal(m1[1], m2[1])
+
+
+@pytest.mark.parametrize("name,K", [("mx_case3_32768x128x112", 512), ("per_token_int32_4096x64x64", 256)])
+def test_host_pipeline_chunks_match_device_call(name, K):
+    # the chunked three-stream pipeline from pinned host memory gives the bytes of one
+    # device call, also on a second step that reuses its buffers
+    w = WORKLOADS[name].with_tokens(K)
+    x, P1, P2 = make_inputs(w, seed=5)
+    fq = FlatQuant(w.K, w.M, w.N)
+    xd, P1d, P2d = x.cuda(), P1.cuda(), P2.cuda()
+    if w.mode == "mx":
+        ref = fq.quantize_mx(xd, P1d, P2d, w.dst_type_max)
+    else:
+        ref = fq.quantize_per_token(xd, P1d, P2d, w.clip_ratio, w.out)
+    for chunks in (8, 1):
+        pipe = HostPipeline(fq, w.mode, w.out if w.mode == "per_token" else "int4", chunks=chunks)
+        oh, sh = pipe.host_outputs()
+        for _ in range(2):
+            oh.zero_()
+            sh.zero_()
+            pipe.run(x.pin_memory(), P1.pin_memory(), P2.pin_memory(), oh, sh,
+                     clip_ratio=w.clip_ratio, dst_type_max=w.dst_type_max)
+            torch.cuda.synchronize()
+            assert torch.equal(oh, ref[0].cpu()) and torch.equal(sh, ref[1].cpu())
 
 
 def test_invalid_arguments_return_page_codes():
