@@ -158,6 +158,16 @@ FQ_API fq_kernel fq_last_kernel(const fq_handle *h);
 /* Number of kernel launches the last successful call on h made. */
 FQ_API int fq_last_launch_count(const fq_handle *h);
 
+/* Test hook for the failure path (the page has no counterpart). Arms the handle so that
+ * its next tensor-core launch issues no x loads and gives every bounded wait a limit of
+ * wait_limit_s seconds (0 < wait_limit_s <= 10): the first stage-A wait can then only end
+ * by running out, after which the kernel sets the abort flag and a status bit, lets every
+ * role leave its loop, frees its TMEM and returns (the outputs of that call are
+ * undefined). fq_device_status then reports the expiry, and the next call runs normally.
+ * One-shot; calls that take the general kernel ignore it. Returns FQ_ERR_NULLPTR or
+ * FQ_ERR_INVALID for a bad argument. */
+FQ_API fq_status fq_debug_arm_stall(fq_handle *h, double wait_limit_s);
+
 /* Reads and clears the handle's device status word: 0 when no kernel gave up a bounded
  * wait since the last read, else a nonzero code naming the wait (and the call returns
  * FQ_ERR_DEVICE_TIMEOUT). Synchronizes the device. */

@@ -66,6 +66,11 @@ class FlatQuant:
         _lib.check(self._lib.fq_set_kernel(self._h, code), "fq_set_kernel")
         self.kernel = kernel
 
+    def debug_arm_stall(self, wait_limit_s):
+        """Test hook: the next tensor-core launch issues no x loads and every bounded wait in
+        it gives up after wait_limit_s seconds (see fq_debug_arm_stall)."""
+        _lib.check(self._lib.fq_debug_arm_stall(self._h, float(wait_limit_s)), "fq_debug_arm_stall")
+
     @property
     def last_kernel(self):
         return {0: "auto", 1: "general", 2: "tcgen05"}[self._lib.fq_last_kernel(self._h)]

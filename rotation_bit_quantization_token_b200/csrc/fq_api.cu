@@ -24,6 +24,8 @@ struct fq_handle {
   fq_kernel last;
   int last_launches;
   uint32_t* d_status;  // 256-byte device block; word 0 = status
+  uint64_t debug_timeout_ns;  // one-shot test hook for the next tensor-core launch
+  int debug_stall;
 };
 
 namespace {
@@ -75,6 +77,9 @@ fq_status launch(fq_handle* h, int mode, const void* x, const void* P1, const vo
     p.x = x; p.P1 = P1; p.P2 = P2; p.K = h->K; p.M = h->M; p.N = h->N; p.mode = mode;
     p.clip_ratio = clip; p.rule = rule; p.out = out; p.quant_scale = qs; p.scales = scales;
     p.x2 = x2; p.status = h->d_status;
+    p.timeout_ns = h->debug_timeout_ns; p.stall_loads = h->debug_stall;
+    h->debug_timeout_ns = 0;
+    h->debug_stall = 0;
     cudaError_t e = fq::launch_tc(p, fp16_in, h->num_sms, s);
     if (e != cudaSuccess) return cuda_fail(e);
     h->last = FQ_KERNEL_TCGEN05;
@@ -198,6 +203,14 @@ fq_status fq_set_kernel(fq_handle* h, fq_kernel kernel) {
 fq_kernel fq_last_kernel(const fq_handle* h) { return h ? h->last : FQ_KERNEL_AUTO; }
 
 int fq_last_launch_count(const fq_handle* h) { return h ? h->last_launches : 0; }
+
+fq_status fq_debug_arm_stall(fq_handle* h, double wait_limit_s) {
+  if (h == nullptr) return FQ_ERR_NULLPTR;
+  if (!(wait_limit_s > 0.0 && wait_limit_s <= 10.0)) return FQ_ERR_INVALID;
+  h->debug_timeout_ns = uint64_t(wait_limit_s * 1e9);
+  h->debug_stall = 1;
+  return FQ_OK;
+}
 
 fq_status fq_device_status(fq_handle* h, uint32_t* status) {
   if (h == nullptr || status == nullptr) return FQ_ERR_NULLPTR;

@@ -45,6 +45,8 @@ struct TcParams {
   uint8_t* scales;
   float* x2;
   uint32_t* status;    // device status word (bounded waits)
+  uint64_t timeout_ns; // limit of every bounded wait; 0 = the default (4 s)
+  int stall_loads;     // test hook: the producer issues no x loads (see fq_debug_arm_stall)
 };
 
 bool tc_supported(int64_t K, int M, int N);

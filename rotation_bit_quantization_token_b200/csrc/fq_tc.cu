@@ -57,7 +57,7 @@ constexpr int kThreads = 512;  // four warpgroups
 constexpr int kEpi = 3;  // epilogue warpgroups (warps 0-11)
 constexpr int kLaunchRegs = 128, kEpiRegs = 152, kLowRegs = 56;
 static_assert(128 * (kEpi * kEpiRegs + kLowRegs) <= kThreads * kLaunchRegs, "register split");
-constexpr uint64_t kTimeoutNs = 4000000000ull;  // 4 s: far beyond any legitimate wait
+constexpr uint64_t kTimeoutNs = 4000000000ull;  // 4 s: far beyond any legitimate wait (default)
 
 // status bits (device status word)
 enum : uint32_t {
@@ -111,6 +111,7 @@ struct Bars {
   uint64_t mma_done[2];
   uint32_t tmem_base;
   int abort;
+  uint64_t timeout_ns;  // limit of every bounded wait of this launch
   int group_exit[kEpi][2];  // per epilogue group: exit decision, one slot per use parity
   float red[kEpi][4];
   float wmax[kThreads / 32];
@@ -363,7 +364,7 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, Bar
   for (;;) {
     if (mbar_try_wait(b, parity)) return true;
     if (*reinterpret_cast<volatile int*>(&bars->abort)) return false;
-    if (globaltimer() - t0 > kTimeoutNs) {
+    if (globaltimer() - t0 > bars->timeout_ns) {
       *reinterpret_cast<volatile int*>(&bars->abort) = 1;
       atomicOr(status, code);
       return false;
@@ -446,6 +447,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     mbar_init(&bars->mma_done[0], 1);
     mbar_init(&bars->mma_done[1], 1);
     bars->abort = 0;
+    bars->timeout_ns = p.timeout_ns != 0 ? p.timeout_ns : kTimeoutNs;
     for (int g = 0; g < kEpi; ++g) bars->group_exit[g][0] = bars->group_exit[g][1] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -529,7 +531,9 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
   if (warp == 12) {
     // ---------------- TMA producer ----------------
     setmaxnreg_dec<kLowRegs>();
-    if (lane == 0) {
+    // (test hook) with stall_loads the producer issues nothing, so the first stage-A wait can
+    // only end by running out
+    if (lane == 0 && !p.stall_loads) {
       int i = 0;
       int last_i[kStages];
 #pragma unroll
@@ -550,7 +554,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
         const uint32_t b = smem_u32(&bars->x_full[s]);
         const uint64_t t0 = globaltimer();
         while (!mbar_try_wait(b, (last_i[s] / kStages) & 1)) {
-          if (globaltimer() - t0 > kTimeoutNs) { atomicOr(p.status, kStDrain); break; }
+          if (globaltimer() - t0 > bars->timeout_ns) { atomicOr(p.status, kStDrain); break; }
         }
       }
     }
@@ -630,7 +634,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       const uint32_t bd = smem_u32(&bars->mma_done[mb]);
       const uint64_t t0 = globaltimer();
       while (!mbar_try_wait(bd, 0)) {
-        if (globaltimer() - t0 > kTimeoutNs) { atomicOr(p.status, kStMmaDone); break; }
+        if (globaltimer() - t0 > bars->timeout_ns) { atomicOr(p.status, kStMmaDone); break; }
       }
     }
     __syncwarp();
