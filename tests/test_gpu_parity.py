@@ -118,7 +118,8 @@ def test_host_example_fp16_closed_form():
 
 @pytest.mark.parametrize("shape", [(1, 16, 16), (3, 3, 14), (5, 1, 96), (4, 17, 2),
                                    (6, 48, 40), (3, 256, 256), (9, 64, 64), (5, 128, 112),
-                                   (3, 32, 64), (7, 64, 80)])
+                                   (3, 32, 64), (7, 64, 80), (4, 32, 96), (3, 128, 128),
+                                   (5, 128, 64), (6, 32, 128), (2, 64, 96), (4, 128, 80)])
 @pytest.mark.parametrize("mode", ["per_token", "mx0", "mx6", "mx7", "mx10"])
 def test_edge_shapes(shape, mode):
     K, M, N = shape
@@ -128,6 +129,22 @@ def test_edge_shapes(shape, mode):
     else:
         w = Workload("edge", K, M, N, "mx", "normal_outliers", dst_type_max=float(mode[2:]))
     x, P1, P2 = make_inputs(w, seed=K * 1000 + M * 10 + N)
+    for kernel in _kernels_for(w):
+        _run_and_compare(w, x, P1, P2, kernel)
+
+
+@pytest.mark.parametrize("shape", [(5, 128, 112), (7, 64, 64), (3, 32, 96)])
+@pytest.mark.parametrize("mode", ["per_token", "mx10"])
+def test_fp16_inputs_tensor_core_shapes(shape, mode):
+    # fp16 x, P1, P2 (the page's second input type) on the shapes the tensor-core kernel takes
+    K, M, N = shape
+    from rotation_bit_quantization_token_b200.workloads import Workload
+    if mode == "per_token":
+        w = Workload("fp16", K, M, N, "per_token", "normal", out="int4", clip_ratio=1.0)
+    else:
+        w = Workload("fp16", K, M, N, "mx", "normal_outliers", dst_type_max=10.0)
+    x, P1, P2 = make_inputs(w, seed=11, dtype=torch.float16)
+    assert x.dtype == torch.float16
     for kernel in _kernels_for(w):
         _run_and_compare(w, x, P1, P2, kernel)
 
