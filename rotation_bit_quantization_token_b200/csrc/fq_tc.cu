@@ -19,20 +19,20 @@
 // range, converted to fp16 and transposed to K-major once per CTA. The powers of two
 // are undone exactly in the epilogue.
 //
-// Roles (one CTA per SM, persistent over tiles, 512 threads = 4 warpgroups):
-//   warps 0-11  three epilogue warpgroups; group g takes the local tiles i = g (mod 3):
-//               it reads Y from TMEM (lane = row), scales each row by a power of two and
-//               writes fp16 hi / lo back into the same TMEM columns for stage B; then it
-//               reads the row of X'' in one round trip, releases the buffer, forms
-//               per-token or per-group scales and codes, stages them in shared memory and
-//               stores them with bulk copies
-//   warp 12     TMA producer: x tiles (128 rows x N, 128B-swizzled) into a 4-stage ring
-//   warp 13     MMA issuer of stage A (A = BD(P1) in SMEM, B = x tile, MN-major); it
-//               also owns the TMEM allocation
-//   warp 14     MMA issuer of stage B (A = hi/lo Y in TMEM, B = P2^T in SMEM)
-//   warp 15     idle after the prologue
-// TMEM holds two to four D_A slots (Y, then its hi / lo) and two or three D_B slots (X''),
-// as many as fit in 512 columns, so stage A runs ahead of the epilogue.
+// Roles (one CTA per SM, persistent over tiles, 640 threads = 5 warpgroups):
+//   warps 0-15  four epilogue warpgroups; group g takes the local tiles i = g (mod 4): it
+//               reads Y from TMEM (lane = row), scales each row by a power of two and writes
+//               fp16 hi / lo back into the same TMEM columns for stage B; then it reads the
+//               row of X'' (twice: block maxima, then the codes, so that a thread never
+//               holds a whole row), releases the buffer, forms per-token or per-group scales
+//               and codes, stages them in shared memory and stores them with bulk copies
+//   warp 16     TMA producer: x tiles (128 rows x N, 128B-swizzled) into a 3- or 4-stage ring
+//   warp 17     MMA issuer of stage A (A = BD(P1) in TMEM, or in SMEM when N = 128; B = x
+//               tile, MN-major); it also owns the TMEM allocation
+//   warp 18     MMA issuer of stage B (A = hi/lo Y in TMEM, B = P2^T in SMEM)
+//   warp 19     idle after the prologue
+// TMEM holds D_A slots (Y, then its hi / lo) and D_B slots (X''), two of each for N >= 96,
+// so stage A of the next tile runs while an epilogue group still encodes this one.
 // Every wait is bounded in time; on expiry the kernel records a code in the status word,
 // drains its copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -42,6 +42,7 @@
 
 #include <cstdint>
 #include <mutex>
+#include <type_traits>
 
 #include "fq_internal.h"
 #include "fq_quant.cuh"
@@ -49,13 +50,14 @@
 namespace fq {
 namespace {
 
-constexpr int kStages = 4;
-constexpr int kThreads = 512;  // four warpgroups
-// Register split (setmaxnreg): launched at kLaunchRegs per thread; the three epilogue
+constexpr int kStagesMax = 4;
+constexpr int kThreads = 640;  // five warpgroups
+// Register split (setmaxnreg): launched at kLaunchRegs per thread; the four epilogue
 // warpgroups rise to kEpiRegs and the producer / MMA warpgroup drops to kLowRegs. The shares add up to no more than the registers the block was
 // launched with, so setmaxnreg.inc always finds what it asks for.
-constexpr int kEpi = 3;  // epilogue warpgroups (warps 0-11)
-constexpr int kLaunchRegs = 128, kEpiRegs = 152, kLowRegs = 56;
+constexpr int kEpi = 4;  // epilogue warpgroups (warps 0-15)
+constexpr int kLaunchRegs = 96, kEpiRegs = 104, kLowRegs = 56;
+constexpr int kWarpProducer = 16, kWarpMmaA = 17, kWarpMmaB = 18;
 static_assert(128 * (kEpi * kEpiRegs + kLowRegs) <= kThreads * kLaunchRegs, "register split");
 constexpr uint64_t kTimeoutNs = 4000000000ull;  // 4 s: far beyond any legitimate wait (default)
 
@@ -71,6 +73,8 @@ struct Geo {
   static_assert(N % 16 == 0 && N >= 64 && N <= 128, "tensor-core kernel covers N in [64,128], N % 16 == 0");
   static constexpr int kAtoms = (N + 63) / 64;              // 64-element swizzle atoms along N
   static constexpr int kXStage = kAtoms * 128 * 128;        // bytes per x stage
+  // x ring depth: four stages, three at N = 128 where BD(P1) stays in shared memory
+  static constexpr int kStages = N == 128 ? 3 : 4;
   // BD(P1) sits in TMEM (64 columns; stage A is then a TS MMA that reads only the x tile
   // from shared memory, 3.5 KB instead of 7.5 KB per MMA at N = 112) when four N-column
   // slots still fit beside it; otherwise in shared memory, 128 x 128, two K atoms (SS).
@@ -100,8 +104,8 @@ struct Geo {
 };
 
 struct Bars {
-  uint64_t x_full[kStages];
-  uint64_t x_empty[kStages];
+  uint64_t x_full[kStagesMax];
+  uint64_t x_empty[kStagesMax];
   // Every barrier below is waited for by one thread or one warpgroup, phase after phase.
   uint64_t da_full[kEpi];   // stage A of tile i done (barrier of its epilogue group i % kEpi)
   uint64_t db_full[kEpi];   // stage B of tile i done (same)
@@ -431,7 +435,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
   lmax = warp_max(lmax);
   if (lane == 0) bars->wmax[warp] = lmax;
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < G::kStages; ++s) {
       mbar_init(&bars->x_full[s], 1);
       mbar_init(&bars->x_empty[s], 1);
     }
@@ -496,7 +500,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     }
   }
   fence_proxy_async();
-  if (warp == 13) tmem_alloc(&bars->tmem_base, G::kTmemCols);
+  if (warp == kWarpMmaA) tmem_alloc(&bars->tmem_base, G::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -528,19 +532,19 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     tc_fence_after();
   }
 
-  if (warp == 12) {
+  if (warp == kWarpProducer) {
     // ---------------- TMA producer ----------------
     setmaxnreg_dec<kLowRegs>();
     // (test hook) with stall_loads the producer issues nothing, so the first stage-A wait can
     // only end by running out
     if (lane == 0 && !p.stall_loads) {
       int i = 0;
-      int last_i[kStages];
+      int last_i[G::kStages];
 #pragma unroll
-      for (int s = 0; s < kStages; ++s) last_i[s] = -1;
+      for (int s = 0; s < G::kStages; ++s) last_i[s] = -1;
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
-        const int s = i % kStages;
-        if (!wait_bounded(&bars->x_empty[s], ((i / kStages) & 1) ^ 1, bars, p.status, kStProducerEmpty)) break;
+        const int s = i % G::kStages;
+        if (!wait_bounded(&bars->x_empty[s], ((i / G::kStages) & 1) ^ 1, bars, p.status, kStProducerEmpty)) break;
         mbar_arrive_expect_tx(&bars->x_full[s], G::kXStage);
 #pragma unroll
         for (int a = 0; a < G::kAtoms; ++a)
@@ -549,16 +553,16 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
         last_i[s] = i;
       }
       // drain: every issued load has landed before the CTA may exit
-      for (int s = 0; s < kStages; ++s) {
+      for (int s = 0; s < G::kStages; ++s) {
         if (last_i[s] < 0) continue;
         const uint32_t b = smem_u32(&bars->x_full[s]);
         const uint64_t t0 = globaltimer();
-        while (!mbar_try_wait(b, (last_i[s] / kStages) & 1)) {
+        while (!mbar_try_wait(b, (last_i[s] / G::kStages) & 1)) {
           if (globaltimer() - t0 > bars->timeout_ns) { atomicOr(p.status, kStDrain); break; }
         }
       }
     }
-  } else if (warp == 13 || warp == 14) {
+  } else if (warp == kWarpMmaA || warp == kWarpMmaB) {
     // ---------------- MMA issuers ----------------
     // Warp 13 issues stage A of every tile, warp 14 stage B, each in tile order and each
     // with blocking waits (a waiting warp takes no issue slots from the epilogue warps on
@@ -574,13 +578,13 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     // waits for the epilogue to read tile i out.
     setmaxnreg_dec<kLowRegs>();
     const int n_local = (blockIdx.x < num_tiles) ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    const int mb = warp - 13;
+    const int mb = warp - kWarpMmaA;
     if (mb == 0) {
       constexpr uint32_t kIdA = idesc_f16(!kF16, !kF16, true, N);
       const uint64_t p1_desc = desc64(sbase + G::kOffP1, 16);
       for (int a = 0; a < n_local; ++a) {
-        const int s = a % kStages, sa = a % G::kNA;
-        if (!warp_wait(&bars->x_full[s], (a / kStages) & 1, bars, p.status, kStMmaXFull)) break;
+        const int s = a % G::kStages, sa = a % G::kNA;
+        if (!warp_wait(&bars->x_full[s], (a / G::kStages) & 1, bars, p.status, kStMmaXFull)) break;
         if (a >= G::kNA && !warp_wait(&bars->da_free[sa], ((a / G::kNA) - 1) & 1, bars, p.status, kStMmaTmemEmpty))
           break;
         tc_fence_after();
@@ -638,7 +642,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       }
     }
     __syncwarp();
-  } else if (warp == 15) {
+  } else if (warp == kWarpMmaB + 1) {
     setmaxnreg_dec<kLowRegs>();  // idle warp of the producer / MMA warpgroup
   } else {
     // ---------------- epilogue warpgroups: split, then quantize, the same tile ----------------
@@ -646,8 +650,10 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     // (D_A) into fp16 hi / lo for stage B, publishing each pair of 16-column blocks as
     // soon as it is in TMEM, then waits for stage B and turns X'' (D_B) into codes and
     // scales. A thread owns one row (TMEM lane) throughout, so its row exponent stays in
-    // a register. The groups work on consecutive tiles at the same time, so the split of
-    // one tile overlaps the split and the encoding of the next ones.
+    // a register. Both phases read their row from TMEM twice (maxima first, then the
+    // values again for the conversion or the codes), so a thread never holds a whole row:
+    // that keeps four groups within the registers of 640 threads, and reads from TMEM do
+    // not slow the MMAs.
     setmaxnreg_inc<kEpiRegs>();
     const int eg = warp >> 2;              // group: tile residue and staging buffer
     const int q = warp & 3;                // TMEM lane quarter of this warp
@@ -660,6 +666,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     uint8_t* s_out = smem + G::kOffOut + eg * G::kOutStride;
     const uint32_t s_out_u32 = sbase + G::kOffOut + eg * G::kOutStride;
     constexpr int NS = N / 16;                 // 16-column segments
+    constexpr int kB1 = (NS + 1) / 2, kB2 = NS - kB1;  // the two batches of a row, in blocks
 
     int jj = 0;  // tiles done by this group
     for (int i = eg, tile = blockIdx.x + eg * gridDim.x; tile < num_tiles;
@@ -679,52 +686,60 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       bool ok = warp_wait(&bars->da_full[eg], jj & 1, bars, p.status, kStEpiAFull);
       if (ok) {
         tc_fence_after();
-        // the row comes out of TMEM in two batches; the maximum of the first is formed
-        // while the second is in flight
-        constexpr int kB1 = (G::kBlocks + 1) / 2;
-        float y[N];
+        // pass 1: the row maximum, in two batches
+        float m;
+        {
+          float y[kB1 * 16];
 #pragma unroll
-        for (int c = 0; c < kB1; ++c) tmem_ld16(t_lane + colA + c * 16, y + c * 16);
-        tmem_wait_ld();
+          for (int c = 0; c < kB1; ++c) tmem_ld16(t_lane + colA + c * 16, y + c * 16);
+          tmem_wait_ld();
+          m = absmax<kB1 * 16>(y);
+        }
+        {
+          float y[kB2 * 16];
 #pragma unroll
-        for (int c = kB1; c < G::kBlocks; ++c) tmem_ld16(t_lane + colA + c * 16, y + c * 16);
-        const float m1 = absmax<kB1 * 16>(y);
-        tmem_wait_ld();
-        s_exp = prescale_exp(fmaxf(m1, absmax<N - kB1 * 16>(y + kB1 * 16)));
+          for (int c = 0; c < kB2; ++c) tmem_ld16(t_lane + colA + (kB1 + c) * 16, y + c * 16);
+          tmem_wait_ld();
+          m = fmaxf(m, absmax<kB2 * 16>(y));
+        }
+        s_exp = prescale_exp(m);
         const float sc = exp2i(s_exp);
         const float2 sc2 = make_float2(sc, sc);
-        // each 16-column block of the row becomes 8 words of hi then 8 words of lo; every
-        // pair of blocks is published on its own barrier as soon as its stores have
-        // landed, and the next pair is converted while they are in flight
-        auto convert = [&](int c, uint32_t* hl) {
+        // pass 2: each pair of 16-column blocks comes out of TMEM again (the next pair is
+        // loaded while this one is converted), becomes 8 words of hi then 8 words of lo per
+        // block, and is published on its own barrier as soon as its stores have landed
+        float ya[32], yb[32];
+        auto load_pair = [&](int g, float* y) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float2 v = __fmul2_rn(make_float2(y[c * 16 + 2 * e], y[c * 16 + 2 * e + 1]), sc2);
-            const __half2 h = __float22half2_rn(v);
-            hl[e] = h2_bits(h);
-            hl[8 + e] = h2_bits(__float22half2_rn(residual2(h, v)));
-          }
+          for (int c = 0; c < 2; ++c)
+            if (2 * g + c < NS) tmem_ld16(t_lane + colA + (2 * g + c) * 16, y + c * 16);
         };
-        uint32_t hl[2][2][16];  // [pair parity][block of the pair][words]
-        convert(0, hl[0][0]);
-        if (G::kBlocks > 1) convert(1, hl[0][1]);
-        tmem_st16(t_lane + colA, hl[0][0]);
-        if (G::kBlocks > 1) tmem_st16(t_lane + colA + 16, hl[0][1]);
+        load_pair(0, ya);
+        tmem_wait_ld();
 #pragma unroll
         for (int g = 0; g < G::kGroups; ++g) {
-          const int nx = (g + 1) & 1;
-          if (g + 1 < G::kGroups) {
-            convert(2 * g + 2, hl[nx][0]);
-            if (2 * g + 3 < G::kBlocks) convert(2 * g + 3, hl[nx][1]);
+          float* cur = (g & 1) ? yb : ya;
+          float* nxt = (g & 1) ? ya : yb;
+          if (g + 1 < G::kGroups) load_pair(g + 1, nxt);
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            if (2 * g + c < NS) {
+              uint32_t hl[16];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float2 v = __fmul2_rn(make_float2(cur[c * 16 + 2 * e], cur[c * 16 + 2 * e + 1]), sc2);
+                const __half2 hv = __float22half2_rn(v);
+                hl[e] = h2_bits(hv);
+                hl[8 + e] = h2_bits(__float22half2_rn(residual2(hv, v)));
+              }
+              tmem_st16(t_lane + colA + (2 * g + c) * 16, hl);
+            }
           }
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars->ys_full[sa][g]);
-          if (g + 1 < G::kGroups) {
-            tmem_st16(t_lane + colA + (2 * g + 2) * 16, hl[nx][0]);
-            if (2 * g + 3 < G::kBlocks) tmem_st16(t_lane + colA + (2 * g + 3) * 16, hl[nx][1]);
-          }
+          if (g + 1 < G::kGroups) tmem_wait_ld();
         }
       } else {
         // a failed wait still publishes every group, so the MMA issuer is not left waiting
@@ -734,47 +749,104 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
           for (int g = 0; g < G::kGroups; ++g) mbar_arrive(&bars->ys_full[sa][g]);
       }
 
-      // keeps the compiler from moving work of one phase into the other, which would
-      // hold both rows in registers at once
+      // keeps the compiler from moving work of one phase into the other
       asm volatile("" ::: "memory");
       // ---- quantize: X'' = D * 2^crow -> codes and scales ----
-      // D_B of tile i is free again for stage B of tile i + NB as soon as this group has
-      // read it, so the whole row comes out of TMEM in one round trip first.
       // phase jj of this group's stage-B barrier; stage B of tile i + kEpi cannot complete
       // before this group has read D_B out (see the MMA issuers)
       const uint32_t colB = uint32_t((G::kNA + sb) * N);
       ok = ok && warp_wait(&bars->db_full[eg], jj & 1, bars, p.status, kStEpiBFull);
-      float d[N];
-      if (ok) {
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < NS; ++c) tmem_ld16(t_lane + colB + c * 16, d + c * 16);
-        tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int e = 0; e < N; ++e) d[e] = 0.0f;
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->tm_empty[sb]);
       const int crow = -(s_exp + t_exp);
       const float fcrow = exp2i(crow);
+      // codes (or x'' in rotate mode) of blocks [c0, c0 + nbk), read again from TMEM
+      auto block_pass = [&](auto nbk_c, int c0, const float* Fseg) {
+        constexpr int nbk = decltype(nbk_c)::value;
+        float d[nbk * 16];
+        if (ok) {
+#pragma unroll
+          for (int c = 0; c < nbk; ++c) tmem_ld16(t_lane + colB + (c0 + c) * 16, d + c * 16);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < nbk * 16; ++e) d[e] = 0.0f;
+        }
+        if constexpr (kMode == kModeRotate) {
+          if (row_valid) {
+            float4* dst = reinterpret_cast<float4*>(p.x2 + grow * N + c0 * 16);
+#pragma unroll
+            for (int e = 0; e < nbk * 16; e += 4)
+              dst[e / 4] = make_float4(d[e] * fcrow, d[e + 1] * fcrow, d[e + 2] * fcrow, d[e + 3] * fcrow);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < nbk; ++c) {
+            const int sg = c0 + c;
+            const float2 F2 = make_float2(Fseg[sg], Fseg[sg]);
+            uint32_t words[2];
+#pragma unroll
+            for (int wd = 0; wd < 2; ++wd) {
+              const float* w = d + c * 16 + wd * 8;
+              if constexpr (kMode == kModePerToken) {
+                const float2 magic = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+                uint32_t acc = 0u;
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                  float2 t = __fmul2_rn(make_float2(w[e], w[e + 1]), F2);
+                  t.x = fminf(fmaxf(t.x, -8.0f), 7.0f);
+                  t.y = fminf(fmaxf(t.y, -8.0f), 7.0f);
+                  // adding 1.5 * 2^23 rounds to an integer (half to even) held in the low bits
+                  const float2 u = __fadd2_rn(t, magic);
+                  acc = bfi4(__float_as_uint(u.x), acc, 4 * e);
+                  acc = bfi4(__float_as_uint(u.y), acc, 4 * e + 4);
+                }
+                words[wd] = acc;
+              } else {
+                const float2 a = __fmul2_rn(make_float2(w[0], w[1]), F2);
+                const float2 b = __fmul2_rn(make_float2(w[2], w[3]), F2);
+                const float2 cc = __fmul2_rn(make_float2(w[4], w[5]), F2);
+                const float2 dd = __fmul2_rn(make_float2(w[6], w[7]), F2);
+                words[wd] = e2m1_canonical_zero(e2m1x8(a, b, cc, dd));
+              }
+            }
+            *reinterpret_cast<uint2*>(s_out + row * (N / 2) + sg * 8) = make_uint2(words[0], words[1]);
+          }
+        }
+      };
+      if (ok) tc_fence_after();
 
       if constexpr (kMode == kModeRotate) {
-        if (row_valid) {
-          float4* dst = reinterpret_cast<float4*>(p.x2 + grow * N);
-#pragma unroll
-          for (int e = 0; e < N; e += 4)
-            dst[e / 4] = make_float4(d[e] * fcrow, d[e + 1] * fcrow, d[e + 2] * fcrow, d[e + 3] * fcrow);
-        }
+        block_pass(std::integral_constant<int, kB1>(), 0, nullptr);
+        block_pass(std::integral_constant<int, kB2>(), kB1, nullptr);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->tm_empty[sb]);
         if (leader) bars->group_exit[eg][jj & 1] = *reinterpret_cast<volatile int*>(&bars->abort) | int(!ok);
         named_bar(bar_id, 128);
         if (bars->group_exit[eg][jj & 1]) break;
         continue;
       } else {
+        // pass 1: the maximum of each 16-column block, in two batches
         float smax[NS];
 #pragma unroll
-        for (int sg = 0; sg < NS; ++sg) smax[sg] = absmax16(d + sg * 16);
+        for (int sg = 0; sg < NS; ++sg) smax[sg] = 0.0f;
+        if (ok) {
+          {
+            float d[kB1 * 16];
+#pragma unroll
+            for (int c = 0; c < kB1; ++c) tmem_ld16(t_lane + colB + c * 16, d + c * 16);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < kB1; ++c) smax[c] = absmax16(d + c * 16);
+          }
+          {
+            float d[kB2 * 16];
+#pragma unroll
+            for (int c = 0; c < kB2; ++c) tmem_ld16(t_lane + colB + (kB1 + c) * 16, d + c * 16);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < kB2; ++c) smax[kB1 + c] = absmax16(d + c * 16);
+          }
+        }
         if (leader) bulk_wait_read<0>();  // this group's previous store has left the staging buffer
         float Fseg[NS];
         if constexpr (kMode == kModePerToken) {
@@ -831,38 +903,13 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
             }
           }
         }
-        // codes: 16 columns (2 words) at a time into the staging buffer
-#pragma unroll
-        for (int sg = 0; sg < NS; ++sg) {
-          const float2 F2 = make_float2(Fseg[sg], Fseg[sg]);
-          uint32_t words[2];
-#pragma unroll
-          for (int wd = 0; wd < 2; ++wd) {
-            const float* w = d + sg * 16 + wd * 8;
-            if constexpr (kMode == kModePerToken) {
-              const float2 magic = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
-              uint32_t acc = 0u;
-#pragma unroll
-              for (int e = 0; e < 8; e += 2) {
-                float2 t = __fmul2_rn(make_float2(w[e], w[e + 1]), F2);
-                t.x = fminf(fmaxf(t.x, -8.0f), 7.0f);
-                t.y = fminf(fmaxf(t.y, -8.0f), 7.0f);
-                // adding 1.5 * 2^23 rounds to an integer (half to even) held in the low bits
-                const float2 u = __fadd2_rn(t, magic);
-                acc = bfi4(__float_as_uint(u.x), acc, 4 * e);
-                acc = bfi4(__float_as_uint(u.y), acc, 4 * e + 4);
-              }
-              words[wd] = acc;
-            } else {
-              const float2 a = __fmul2_rn(make_float2(w[0], w[1]), F2);
-              const float2 b = __fmul2_rn(make_float2(w[2], w[3]), F2);
-              const float2 cc = __fmul2_rn(make_float2(w[4], w[5]), F2);
-              const float2 dd = __fmul2_rn(make_float2(w[6], w[7]), F2);
-              words[wd] = e2m1_canonical_zero(e2m1x8(a, b, cc, dd));
-            }
-          }
-          *reinterpret_cast<uint2*>(s_out + row * (N / 2) + sg * 8) = make_uint2(words[0], words[1]);
-        }
+        // pass 2: the codes, in the same two batches
+        block_pass(std::integral_constant<int, kB1>(), 0, Fseg);
+        block_pass(std::integral_constant<int, kB2>(), kB1, Fseg);
+        // D_B is free for stage B of tile i + NB
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->tm_empty[sb]);
         fence_proxy_async();
         if (leader) bars->group_exit[eg][jj & 1] = *reinterpret_cast<volatile int*>(&bars->abort) | int(!ok);
         named_bar(bar_id, 128);
@@ -881,7 +928,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 13) {
+  if (warp == kWarpMmaA) {
     tc_fence_after();
     tmem_dealloc(tmem, G::kTmemCols);
   }
