@@ -564,7 +564,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     }
   } else if (warp == kWarpMmaA || warp == kWarpMmaB) {
     // ---------------- MMA issuers ----------------
-    // Warp 13 issues stage A of every tile, warp 14 stage B, each in tile order and each
+    // Warp 17 issues stage A of every tile, warp 18 stage B, each in tile order and each
     // with blocking waits (a waiting warp takes no issue slots from the epilogue warps on
     // its sub-partition). The whole warp runs the loop, so descriptors stay warp-uniform,
     // and one elected lane issues.
