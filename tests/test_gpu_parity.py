@@ -225,6 +225,25 @@ def test_host_pipeline_chunks_match_device_call(name, K):
             assert torch.equal(oh, ref[0].cpu()) and torch.equal(sh, ref[1].cpu())
 
 
+@pytest.mark.parametrize("name", NAMES)
+def test_full_size_repeatable(name):
+    # ten launches at the full size give the same bytes: the pipeline's barriers leave no
+    # room for a race to change the result from one run to the next
+    w = WORKLOADS[name]
+    x, P1, P2 = (t.cuda() for t in make_inputs(w, seed=3))
+    fq = FlatQuant(w.K, w.M, w.N)
+    if w.mode == "mx":
+        run = lambda: fq.quantize_mx(x, P1, P2, w.dst_type_max)  # noqa: E731
+    else:
+        run = lambda: fq.quantize_per_token(x, P1, P2, w.clip_ratio, w.out)  # noqa: E731
+    ref = [t.clone() for t in run()]
+    for _ in range(10):
+        out = run()
+        assert torch.equal(out[0], ref[0]) and torch.equal(out[1], ref[1])
+    torch.cuda.synchronize()
+    assert fq.device_status() == 0
+
+
 def test_invalid_arguments_return_page_codes():
     dev = torch.device("cuda", 0)
     lib = _lib.load()
