@@ -16,7 +16,7 @@ matmul to FP4 E2M1 quantization fusion" (http://www.zwxr.cn/news/277566):
   (8.0-12.0 and other values): groups of 32 consecutive elements of x'' reshaped to
   [K, M*N]; E8M0 shared exponents in a [K, ceilDiv(M*N, 64), 2] tensor; E2M1 codes.
 
-Readings taken where the page is silent or garbled (each is listed in the design doc):
+Readings taken where the page is silent or garbled:
 
 * x'' is formed in float64 with no intermediate rounding.
 * Every step that turns a float into an integer (a code, an exponent) is taken in
