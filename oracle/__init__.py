@@ -10,9 +10,13 @@ quantization fusion" (http://www.zwxr.cn/news/277566), sections "How it works",
 "per-token mode", "per-group mode" cases 1-3, "Parameter quick reference" and
 "Error code quick reference".
 
-Parity unpinned: none. Every public function here is pinned by
-`tests/test_oracle_pins.py` against closed forms, brute force, hand-worked values
-or textbook special cases.
+`consumer.py` restates the dequantization the page says the outputs are emitted for,
+and the FP4 x FP4 contraction that would consume them (no kernel for it exists yet).
+
+Parity unpinned: none. Every public function here is pinned against closed forms,
+brute force, hand-worked values or textbook special cases, by
+`tests/test_oracle_pins.py` (the operator) and `tests/test_oracle_consumer_pins.py`
+(the consumers).
 """
 
 from .flatquant import (  # noqa: F401
@@ -28,4 +32,13 @@ from .flatquant import (  # noqa: F401
     mx_scale_layout,
     flat_quant_per_token,
     flat_quant_mx,
+)
+from .consumer import (  # noqa: F401
+    unpack_nibbles,
+    int4_value,
+    e2m1_value,
+    group_bytes_from_layout,
+    dequantize_per_token,
+    dequantize_mx,
+    mx_matmul,
 )
