@@ -1,0 +1,223 @@
+"""A model of the tensor-core kernel's barrier protocol, run under random interleavings.
+
+This is a host-side check of a design argument, not a test of the CUDA code: the model
+restates, by hand, the waits, arrivals and MMA commits of the roles in
+`rotation_bit_quantization_token_b200/csrc/fq_tc.cu` for one CTA:
+- the TMA producer;
+- the stage-A and stage-B MMA issuers, whose MMAs and commits complete asynchronously but
+  in issue order;
+- four epilogue groups of four warps each, every warp its own actor.
+
+mbarriers follow their parity semantics: a wait for parity P passes while the barrier's
+completed-phase count has the other parity. A random scheduler interleaves the actors, the
+MMA completions and the TMA landings. Every run must end without a deadlock, every wait
+must pass on exactly the completion it means, and every read of an x stage or TMEM slot
+must see the tile it expects. The scheduler re-draws each actor's speed every few dozen
+steps, so that some actors stall while others run ahead. The kernel's comments state the
+argument this checks: every barrier has waiters that take its phases in order, and none is
+ever two phases behind.
+
+Planted mistakes must each be caught, which shows the model can fail:
+- stage B's release of a Y slot left out;
+- a parity off by one;
+- an X'' slot reused without its wait.
+"""
+
+import random
+
+import pytest
+
+
+class Viol(Exception):
+    pass
+
+
+class _Bar:
+    def __init__(self, count):
+        self.count, self.pending, self.done = count, 0, 0
+
+    def arrive(self):
+        self.pending += 1
+        assert self.pending <= self.count
+        if self.pending == self.count:
+            self.pending = 0
+            self.done += 1
+
+
+def run_protocol(T, kNA, kNB, kStages, kGroups, seed, kEpi=4, plant=None):
+    """One CTA over T local tiles. kNA / kNB: TMEM slots of Y and X''; kGroups: pairs of
+    16-column blocks per row. Returns the number of scheduler steps; raises Viol."""
+    rng = random.Random(seed)
+    bars = {}
+
+    def bar(name, count=1):
+        bars[name] = _Bar(count)
+
+    for s in range(kStages):
+        bar(("x_full", s))
+        bar(("x_empty", s))
+    for a in range(4):
+        for g in range(4):
+            bar(("ys_full", a, g), 4)
+        bar(("da_free", a))
+        bar(("tm_empty", a), 4)
+    for e in range(kEpi):
+        bar(("da_full", e))
+        bar(("db_full", e))
+    mem = {}
+
+    def check(buf, want):
+        if mem.get(buf) != want:
+            raise Viol(f"read {buf}: holds {mem.get(buf)}, expected {want}")
+
+    # ops: ("wait", bar, parity, completion meant) | ("arrive", bar) | ("fn", f)
+    #      | ("mma", issuer, f) | ("commit", issuer, bar) | ("tma", stage, tile)
+    def producer():
+        for i in range(T):
+            s = i % kStages
+            yield ("wait", ("x_empty", s), ((i // kStages) & 1) ^ 1, (i // kStages) - 1)
+            yield ("tma", s, i)
+
+    def stage_a():
+        for a in range(T):
+            s, sa = a % kStages, a % kNA
+            yield ("wait", ("x_full", s), (a // kStages) & 1, a // kStages)
+            if a >= kNA:
+                k = (a // kNA) - 1 + (1 if plant == "da_free parity" else 0)
+                yield ("wait", ("da_free", sa), k & 1, k)
+
+            def mma(a=a, s=s, sa=sa):
+                check(("x", s), a)
+                for q in range(4):
+                    mem[("Y", sa, q)] = a
+                    for g in range(kGroups):
+                        mem[("HL", sa, g, q)] = None
+            yield ("mma", "A", mma)
+            yield ("commit", "A", ("x_empty", s))
+            yield ("commit", "A", ("da_full", a % kEpi))
+
+    def stage_b():
+        for b in range(T):
+            sa, sb = b % kNA, b % kNB
+            if b >= kNB and plant != "no tm_empty wait":
+                yield ("wait", ("tm_empty", sb), ((b // kNB) - 1) & 1, (b // kNB) - 1)
+            for g in range(kGroups):
+                yield ("wait", ("ys_full", sa, g), (b // kNA) & 1, b // kNA)
+
+                def mma(b=b, g=g, sa=sa, sb=sb):
+                    for q in range(4):
+                        check(("HL", sa, g, q), b)
+                        mem[("D", sb, q)] = (b, g)
+                yield ("mma", "B", mma)
+            yield ("commit", "B", ("db_full", b % kEpi))
+            if plant != "da_free before stage B":
+                yield ("commit", "B", ("da_free", sa))
+
+    def epilogue_warp(eg, q):
+        jj = 0
+        for i in range(eg, T, kEpi):
+            sa, sb = i % kNA, i % kNB
+            yield ("wait", ("da_full", eg), jj & 1, jj)
+            yield ("fn", lambda i=i, sa=sa: check(("Y", sa, q), i))  # row maximum
+            for g in range(kGroups):
+                yield ("fn", lambda i=i, sa=sa: check(("Y", sa, q), i))  # pair g again
+
+                def split(i=i, g=g, sa=sa):
+                    mem[("HL", sa, g, q)] = i
+                yield ("fn", split)
+                yield ("arrive", ("ys_full", sa, g))
+            yield ("wait", ("db_full", eg), jj & 1, jj)
+            yield ("fn", lambda i=i, sb=sb: check(("D", sb, q), (i, kGroups - 1)))  # maxima
+            yield ("fn", lambda i=i, sb=sb: check(("D", sb, q), (i, kGroups - 1)))  # codes
+            yield ("arrive", ("tm_empty", sb))
+            jj += 1
+
+    actors = {"producer": producer(), "A": stage_a(), "B": stage_b()}
+    for eg in range(kEpi):
+        for q in range(4):
+            actors[("epilogue", eg, q)] = epilogue_warp(eg, q)
+    cur = dict.fromkeys(actors)
+    queues = {"A": [], "B": []}
+    landing = []
+    finished = set()
+    steps = 0
+    while True:
+        steps += 1
+        choices = []
+        for k, gen in actors.items():
+            if k in finished:
+                continue
+            if cur[k] is None:
+                try:
+                    cur[k] = next(gen)
+                except StopIteration:
+                    finished.add(k)
+                    continue
+            op = cur[k]
+            if op[0] == "wait" and (bars[op[1]].done & 1) == op[2]:
+                continue
+            choices.append(("actor", k))
+        choices += [("mma", iss) for iss in queues if queues[iss]]
+        choices += [("tma", j) for j in range(len(landing))]
+        if not choices:
+            if len(finished) == len(actors):
+                return steps
+            raise Viol("deadlock: " + str({k: cur[k][:2] for k in actors if k not in finished}))
+        if steps % 64 == 1:
+            # re-draw every actor's speed now and then, so that some actor stalls for a
+            # while and others run ahead (the orders a uniform choice almost never makes)
+            speed = {c: rng.choice((0.01, 0.1, 1.0, 1.0, 4.0)) for c in
+                     list(actors) + ["q:A", "q:B", "tma"]}
+        weights = [speed[c[1] if c[0] == "actor" else ("q:" + c[1] if c[0] == "mma" else "tma")]
+                   for c in choices]
+        kind, k = rng.choices(choices, weights)[0]
+        if kind == "actor":
+            op, cur[k] = cur[k], None
+            if op[0] == "wait":
+                if op[3] >= 0 and bars[op[1]].done != op[3] + 1:
+                    raise Viol(f"{k}: wait on {op[1]} passed after {bars[op[1]].done} "
+                               f"completions, meant {op[3] + 1}")
+            elif op[0] == "arrive":
+                bars[op[1]].arrive()
+            elif op[0] == "fn":
+                op[1]()
+            elif op[0] in ("mma", "commit"):
+                queues[op[1]].append(op)
+            else:
+                landing.append((op[1], op[2]))
+        elif kind == "mma":
+            op = queues[k].pop(0)
+            if op[0] == "mma":
+                op[2]()
+            else:
+                bars[op[2]].arrive()
+        else:
+            s, i = landing.pop(k)
+            mem[("x", s)] = i
+            bars[("x_full", s)].arrive()
+
+
+# (N, kNA, kNB, kStages, pairs per row) of the kernel's geometry for each N it covers
+SHAPES = [(64, 4, 3, 4, 2), (80, 3, 2, 4, 3), (96, 2, 2, 4, 3), (112, 2, 2, 4, 4), (128, 2, 2, 3, 4)]
+
+
+@pytest.mark.parametrize("N,kNA,kNB,kStages,pairs", SHAPES)
+def test_protocol_has_no_deadlock_phase_slip_or_stale_read(N, kNA, kNB, kStages, pairs):
+    for T in (1, 2, 3, 5, 9, 17):
+        for seed in range(60):
+            run_protocol(T, kNA, kNB, kStages, pairs, seed)
+
+
+@pytest.mark.parametrize("plant", ["da_free before stage B", "da_free parity", "no tm_empty wait"])
+def test_planted_protocol_mistakes_are_caught(plant):
+    caught = False
+    for T in (3, 5, 9, 17):
+        for seed in range(200):
+            try:
+                run_protocol(T, 2, 2, 4, 4, seed, plant=plant)
+            except Viol:
+                caught = True
+                break
+        if caught:
+            break
+    assert caught, f"the model did not catch: {plant}"
