@@ -34,6 +34,39 @@ def _check_input(name, t, dtype=None):
         raise ValueError(f"{name} must have dtype {dtype}, got {t.dtype}")
 
 
+def _check_device(x, **others):
+    """x on the current CUDA device (the plan was made, and its kernels launch, there) and
+    every other tensor beside it."""
+    cur = torch.cuda.current_device()
+    if x.device.index != cur:
+        raise ValueError(f"x is on {x.device} but the current CUDA device is cuda:{cur}; "
+                         "call torch.cuda.set_device first")
+    for name, t in others.items():
+        if t is not None and t.device != x.device:
+            raise ValueError(f"{name} must be on {x.device}, got {t.device}")
+
+
+def _check_output(name, t, nbytes, device, dtype=None):
+    """A caller-supplied output: on `device`, contiguous, exactly `nbytes` bytes (the
+    kernel writes all of them, so a smaller buffer would be overrun), and of `dtype` when
+    the values are numbers rather than packed codes."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must have dtype {dtype}, got {t.dtype}")
+    have = t.numel() * t.element_size()
+    if have != nbytes:
+        raise ValueError(f"{name} must hold {nbytes} bytes, got {have}")
+
+
+def _scale_bytes(K, M, N):
+    return K * (-(-M * N // 64)) * 2
+
+
 class FlatQuant:
     """A plan for one shape [K, M, N] and input dtype (the handle of fq_create)."""
 
@@ -102,6 +135,7 @@ class FlatQuant:
             _check_input("P2", P2, self.dtype)
             if tuple(P2.shape) != (self.N, self.N):
                 raise ValueError("P2 must be [N, N]")
+        _check_device(x, P1=P1, P2=P2)
         return P2
 
     def quantize_per_token(self, x, P1, P2, clip_ratio=1.0, out_dtype="int4",
@@ -115,8 +149,12 @@ class FlatQuant:
                 out = torch.empty((K, M, N // 8), dtype=torch.int32, device=x.device)
             else:
                 out = torch.empty((K, M * N // 2), dtype=torch.uint8, device=x.device)
+        else:
+            _check_output("out", out, K * M * N // 2, x.device)
         if quant_scale is None:
             quant_scale = torch.empty((K,), dtype=torch.float32, device=x.device)
+        else:
+            _check_output("quant_scale", quant_scale, 4 * K, x.device, torch.float32)
         fmt = _lib.FQ_OUT_INT32 if out_dtype == "int32" else _lib.FQ_OUT_INT4
         _lib.check(self._lib.fq_quantize_per_token(
             self._h, _ptr(x), _ptr(P1), _ptr(P2), float(clip_ratio), fmt, _ptr(out),
@@ -130,8 +168,12 @@ class FlatQuant:
         K, M, N = self.K, self.M, self.N
         if out is None:
             out = torch.empty((K, M * N // 2), dtype=torch.uint8, device=x.device)
+        else:
+            _check_output("out", out, K * M * N // 2, x.device)
         if scales is None:
             scales = torch.empty((K, -(-M * N // 64), 2), dtype=torch.uint8, device=x.device)
+        else:
+            _check_output("scales", scales, _scale_bytes(K, M, N), x.device)
         _lib.check(self._lib.fq_quantize_mx(
             self._h, _ptr(x), _ptr(P1), _ptr(P2), float(dst_type_max), _ptr(out),
             _ptr(scales), _stream_ptr(stream)), "fq_quantize_mx")
@@ -142,6 +184,8 @@ class FlatQuant:
         P2 = self._inputs(x, P1, P2, allow_no_p2=True)
         if out is None:
             out = torch.empty((self.K, self.M, self.N), dtype=torch.float32, device=x.device)
+        else:
+            _check_output("out", out, 4 * self.K * self.M * self.N, x.device, torch.float32)
         _lib.check(self._lib.fq_debug_rotate(self._h, _ptr(x), _ptr(P1), _ptr(P2), _ptr(out),
                                              _stream_ptr(stream)), "fq_debug_rotate")
         return out
@@ -170,11 +214,22 @@ def quantize_mx_static(x, P1, P2, dst_type_max=0.0, out=None, scales=None, strea
         P2 = None
     if P2 is not None:
         _check_input("P2", P2, x.dtype)
+    if x.dim() != 3:
+        raise ValueError("x must be [K, M, N]")
     K, M, N = x.shape
+    if tuple(P1.shape) != (M, M):
+        raise ValueError("P1 must be [M, M]")
+    if P2 is not None and tuple(P2.shape) != (N, N):
+        raise ValueError("P2 must be [N, N]")
+    _check_device(x, P1=P1, P2=P2)
     if out is None:
         out = torch.empty((K, M * N // 2), dtype=torch.uint8, device=x.device)
+    else:
+        _check_output("out", out, K * M * N // 2, x.device)
     if scales is None:
         scales = torch.empty((K, -(-M * N // 64), 2), dtype=torch.uint8, device=x.device)
+    else:
+        _check_output("scales", scales, _scale_bytes(K, M, N), x.device)
     _lib.check(lib.fq_quantize_mx_static(K, M, N, _DT[x.dtype], _ptr(x), _ptr(P1), _ptr(P2),
                                          float(dst_type_max), _ptr(out), _ptr(scales),
                                          _stream_ptr(stream)), "fq_quantize_mx_static")

@@ -137,3 +137,29 @@ def test_bench_max_over_ranks_two_gloo_ranks(tmp_path):
     for p, o in zip(procs, outs):
         assert p.returncode == 0, o
         assert "ok" in o
+
+
+def test_output_buffer_checks_on_host():
+    """Caller-supplied outputs are refused before any launch unless they sit on the
+    input's device, are contiguous, hold exactly the bytes the kernel writes, and (for
+    numeric outputs) have the right dtype; an undersized buffer would otherwise be
+    overrun on the GPU. Checked here on CPU tensors, with the CPU as the device."""
+    from rotation_bit_quantization_token_b200 import api
+
+    cpu = torch.device("cpu")
+    K, M, N = 3, 4, 16
+    api._check_output("out", torch.empty((K, M * N // 2), dtype=torch.uint8), K * M * N // 2, cpu)
+    api._check_output("out", torch.empty((K, M, N // 8), dtype=torch.int32), K * M * N // 2, cpu)
+    api._check_output("scales", torch.empty((K, 1, 2), dtype=torch.uint8), api._scale_bytes(K, M, N), cpu)
+    api._check_output("quant_scale", torch.empty(K, dtype=torch.float32), 4 * K, cpu, torch.float32)
+    bad = [
+        (torch.empty((K, M * N // 2 - 1), dtype=torch.uint8), K * M * N // 2, None, "bytes"),
+        (torch.empty((M * N // 2, K), dtype=torch.uint8).t(), K * M * N // 2, None, "contiguous"),
+        (torch.empty(K, dtype=torch.float16), 4 * K, torch.float32, "dtype"),
+        ([0] * K, 4 * K, None, "Tensor"),
+    ]
+    for t, nbytes, dtype, word in bad:
+        with pytest.raises((ValueError, TypeError), match=word):
+            api._check_output("buf", t, nbytes, cpu, dtype)
+    # scale tensor of an odd group count: [K, ceilDiv(M*N, 64), 2] includes the pad slot
+    assert api._scale_bytes(2, 3, 32) == 2 * 2 * 2
