@@ -151,6 +151,16 @@ FQ_API fq_status fq_debug_rotate(fq_handle *h, const void *x, const void *P1, co
  * FQ_ERR_UNSUPPORTED if FQ_KERNEL_TCGEN05 is asked for a shape it does not cover. */
 FQ_API fq_status fq_set_kernel(fq_handle *h, fq_kernel kernel);
 
+/* Intermediate rounding (the page's "How it works" leaves open whether x' = x . P2 is kept
+ * in the input type before P1 . x'; the default keeps it exact). With enable = 1, later
+ * calls on h round every x' element to the handle's 16-bit type (nearest, ties to even)
+ * after summing its products in float32 in index order, then form x'' = P1 . x' from the
+ * rounded values. This is meant for comparison with implementations that store x' so, not
+ * for speed: it runs the general kernel (FQ_ERR_UNSUPPORTED if FQ_KERNEL_TCGEN05 is
+ * selected). enable = 0 restores the default. Returns FQ_ERR_NULLPTR for a null handle and
+ * FQ_ERR_INVALID for enable other than 0 or 1. */
+FQ_API fq_status fq_set_intermediate_rounding(fq_handle *h, int enable);
+
 /* The kernel the last successful call on h launched (FQ_KERNEL_GENERAL or
  * FQ_KERNEL_TCGEN05), or FQ_KERNEL_AUTO before any call. */
 FQ_API fq_kernel fq_last_kernel(const fq_handle *h);

@@ -24,6 +24,8 @@ from .flatquant import (  # noqa: F401
     e2m1_encode,
     e2m1_decode,
     rotate,
+    rotate_rounded,
+    round_to_16bit,
     per_token_quantize,
     pack_nibbles,
     mx_group_view,

@@ -87,6 +87,42 @@ def rotate(x, P1, P2):
     return np.matmul(P1, x1)
 
 
+def round_to_16bit(v, dtype):
+    """float32 values rounded to "bf16" or "fp16" (nearest, ties to even), returned as
+    float64. bf16: the low 16 bits of the float32 encoding are dropped after adding
+    0x7FFF plus the lowest kept bit (round half to even on the bit pattern; finite values
+    only). fp16: numpy's float32 -> float16 cast, which rounds to nearest even."""
+    v = np.asarray(v, dtype=np.float32)
+    if dtype == "fp16":
+        with np.errstate(over="ignore"):
+            return v.astype(np.float16).astype(np.float64)
+    bits = v.view(np.uint32).astype(np.uint64)
+    bits = (bits + 0x7FFF + ((bits >> 16) & 1)) & 0xFFFF0000
+    return bits.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def rotate_rounded(x, P1, P2, dtype="bf16"):
+    """Two-level small matmul with x' kept in the input type between the products: the
+    intermediate-rounding reading of "How it works", whose formulas leave the precision of
+    x' open. Each x'[m, n] is the sum over j = 0, 1, ..., N-1, in that order, of
+    x[m, j] * P2[j, n] in float32: every partial sum is rounded to float32, and the
+    product of two 16-bit inputs is exact in float32. The sum is then rounded to the input
+    type (nearest, ties to even), and x'' = P1 . x' is formed in float64.
+    P2 None or empty skips the right multiply (x' = x, already in the input type)."""
+    x = np.asarray(x, dtype=np.float64)
+    P1 = np.asarray(P1, dtype=np.float64)
+    if P2 is None or np.size(P2) == 0:
+        x1 = x
+    else:
+        x32 = x.astype(np.float32)
+        P2_32 = np.asarray(P2, dtype=np.float32)
+        acc = np.zeros(x.shape, dtype=np.float32)
+        for j in range(x.shape[-1]):
+            acc = (acc + x32[..., j:j + 1] * P2_32[j]).astype(np.float32)
+        x1 = round_to_16bit(acc, dtype)
+    return np.matmul(P1, x1)
+
+
 def per_token_quantize(x2, clip_ratio):
     """Per-token mode (page: "per-token mode"):
     quantScale[k] = max|x''[k]| / (7 / clipRatio) as FLOAT32, out = x'' / quantScale,
@@ -212,12 +248,13 @@ def mx_scale_layout(group_bytes):
     return out.reshape(K, -1, 2)
 
 
-def flat_quant_per_token(x, P1, P2, clip_ratio, out_dtype="int4"):
+def flat_quant_per_token(x, P1, P2, clip_ratio, out_dtype="int4", intermediate=None):
     """Whole per-token path. Returns (out, quantScale, info):
-    out is uint8 [K, M*N/2] for "int4" or int32 [K, M, N/8] for "int32" (same bytes)."""
+    out is uint8 [K, M*N/2] for "int4" or int32 [K, M, N/8] for "int32" (same bytes).
+    intermediate = "bf16" / "fp16" keeps x' in that type (rotate_rounded)."""
     x = np.asarray(x, dtype=np.float64)
     K, M, N = x.shape
-    x2 = rotate(x, P1, P2)
+    x2 = rotate(x, P1, P2) if intermediate is None else rotate_rounded(x, P1, P2, intermediate)
     codes, qscale, v = per_token_quantize(x2, clip_ratio)
     packed = pack_nibbles(codes.reshape(K, M * N))
     if out_dtype == "int32":
@@ -227,12 +264,13 @@ def flat_quant_per_token(x, P1, P2, clip_ratio, out_dtype="int4"):
     return out, qscale, {"x2": x2, "codes": codes, "v": v}
 
 
-def flat_quant_mx(x, P1, P2, dst_type_max):
+def flat_quant_mx(x, P1, P2, dst_type_max, intermediate=None):
     """Whole per-group path. Returns (out uint8 [K, M*N/2], scales uint8
-    [K, ceilDiv(M*N, 64), 2], info)."""
+    [K, ceilDiv(M*N, 64), 2], info). intermediate = "bf16" / "fp16" keeps x' in that
+    type (rotate_rounded)."""
     x = np.asarray(x, dtype=np.float64)
     K, M, N = x.shape
-    x2 = rotate(x, P1, P2)
+    x2 = rotate(x, P1, P2) if intermediate is None else rotate_rounded(x, P1, P2, intermediate)
     codes, gbytes, v, amax = mx_quantize(x2, dst_type_max)
     out = pack_nibbles(codes)
     return out, mx_scale_layout(gbytes), {"x2": x2, "codes": codes, "v": v,

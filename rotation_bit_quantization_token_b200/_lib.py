@@ -32,6 +32,7 @@ _SIGNATURES = {
     "fq_debug_rotate": (_int, [_vp, _vp, _vp, _vp, _vp, _vp]),
     "fq_quantize_mx_static": (_int, [_i64, _i64, _i64, _int, _vp, _vp, _vp, _dbl, _vp, _vp, _vp]),
     "fq_set_kernel": (_int, [_vp, _int]),
+    "fq_set_intermediate_rounding": (_int, [_vp, _int]),
     "fq_debug_arm_stall": (_int, [_vp, _dbl]),
     "fq_last_kernel": (_int, [_vp]),
     "fq_last_launch_count": (_int, [_vp]),

@@ -99,6 +99,13 @@ class FlatQuant:
         _lib.check(self._lib.fq_set_kernel(self._h, code), "fq_set_kernel")
         self.kernel = kernel
 
+    def set_intermediate_rounding(self, enable):
+        """Round x' = x . P2 to the input dtype before the left product (see
+        fq_set_intermediate_rounding); runs the general kernel."""
+        _lib.check(self._lib.fq_set_intermediate_rounding(self._h, int(bool(enable))),
+                   "fq_set_intermediate_rounding")
+        self.intermediate_rounding = bool(enable)
+
     def debug_arm_stall(self, wait_limit_s):
         """Test hook: the next tensor-core launch issues no x loads and every bounded wait in
         it gives up after wait_limit_s seconds (see fq_debug_arm_stall)."""

@@ -26,6 +26,7 @@ struct fq_handle {
   uint32_t* d_status;  // 256-byte device block; word 0 = status
   uint64_t debug_timeout_ns;  // one-shot test hook for the next tensor-core launch
   int debug_stall;
+  int round_x1;  // intermediate rounding of x' (general kernel only)
 };
 
 namespace {
@@ -56,7 +57,7 @@ bool mx_rule_from(double d, fq::MxRule* r) {
 // with bulk copies, so all of them must be 16-byte aligned.
 bool use_tc(const fq_handle* h, const void* x, const void* P1, const void* P2, const void* out,
             const void* scales) {
-  if (h->pref == FQ_KERNEL_GENERAL) return false;
+  if (h->pref == FQ_KERNEL_GENERAL || h->round_x1) return false;
   if (!fq::tc_supported(h->K, h->M, h->N)) return false;
   return aligned(x, 16) && aligned(P1, 16) && (P2 == nullptr || aligned(P2, 16)) &&
          aligned(out, 16) && (scales == nullptr || aligned(scales, 16));
@@ -91,6 +92,7 @@ fq_status launch(fq_handle* h, int mode, const void* x, const void* P1, const vo
   p.x = x; p.P1 = P1; p.P2 = P2; p.K = h->K; p.M = h->M; p.N = h->N; p.mode = mode;
   p.clip_ratio = clip; p.rule = rule; p.out = out; p.quant_scale = qs; p.scales = scales;
   p.x2 = x2;
+  p.round_x1 = h->round_x1;
   cudaError_t e = fq::launch_general(p, fp16_in, general_grid(h), s);
   if (e != cudaSuccess) return cuda_fail(e);
   h->last = FQ_KERNEL_GENERAL;
@@ -197,6 +199,13 @@ fq_status fq_set_kernel(fq_handle* h, fq_kernel kernel) {
   if (kernel == FQ_KERNEL_TCGEN05 && !fq::tc_supported(h->K, h->M, h->N))
     return FQ_ERR_UNSUPPORTED;
   h->pref = kernel;
+  return FQ_OK;
+}
+
+fq_status fq_set_intermediate_rounding(fq_handle* h, int enable) {
+  if (h == nullptr) return FQ_ERR_NULLPTR;
+  if (enable != 0 && enable != 1) return FQ_ERR_INVALID;
+  h->round_x1 = enable;
   return FQ_OK;
 }
 

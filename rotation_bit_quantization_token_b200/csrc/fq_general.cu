@@ -11,8 +11,10 @@
 // The quantizer needs a reduction over the token (per-token absmax) or over groups that
 // may straddle rows and column blocks, so x'' is produced twice: pass 0 reduces, pass 1
 // recomputes the identical values and encodes them. Nothing but the outputs reaches
-// global memory. This kernel serves the small shapes (M, N = 16) and every shape the
-// tensor-core kernel does not cover.
+// global memory. This kernel serves the small shapes (M, N = 16), every shape the
+// tensor-core kernel does not cover, and the intermediate-rounding mode (x' rounded to the
+// input type between the two products, for comparison with implementations that store it
+// so); x' is one float32 FMA chain over j in index order.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cstdint>
@@ -33,6 +35,14 @@ template <>
 __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
 template <>
 __device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
+
+// v rounded to the 16-bit input type (nearest, ties to even) and widened back
+template <typename T>
+__device__ __forceinline__ float round_to(float v);
+template <>
+__device__ __forceinline__ float round_to<__nv_bfloat16>(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
+template <>
+__device__ __forceinline__ float round_to<__half>(float v) { return __half2float(__float2half_rn(v)); }
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -89,7 +99,8 @@ general_kernel(const GeneralParams p) {
             float acc = 0.0f;
             const T* xr = xs + m * N;
             for (int j = 0; j < N; ++j) acc = fmaf(to_f32(xr[j]), p2s[j * kCol + c], acc);
-            xp[o] = acc;
+            // with intermediate rounding, x' is stored in the input type between the products
+            xp[o] = p.round_x1 ? round_to<T>(acc) : acc;
           }
         } else {
           for (int o = tid; o < M * kCol; o += kThreads) {

@@ -24,6 +24,7 @@ struct GeneralParams {
   float* quant_scale;  // [K] per-token
   uint8_t* scales;     // [K, 2*ceilDiv(M*N,64)] per-group
   float* x2;           // [K, M, N] rotate-only
+  int round_x1;        // round x' = x . P2 to the input type (RNE) before the left product
 };
 
 size_t general_smem_bytes(int M, int N, int elem_bytes);

@@ -57,6 +57,7 @@ def test_plan_validation_without_device(lib):
     assert lib.fq_quantize_per_token(None, None, None, None, 1.0, 0, None, None, None) == _lib.FQ_ERR_NULLPTR
     assert lib.fq_destroy(None) == _lib.FQ_OK
     assert lib.fq_last_kernel(None) == 0
+    assert lib.fq_set_intermediate_rounding(None, 1) == _lib.FQ_ERR_NULLPTR
     for code in (0, 161001, 161002, 161003, 161004, 161005):
         assert lib.fq_status_string(code).decode().startswith("FQ_")
 

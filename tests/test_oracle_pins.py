@@ -383,3 +383,50 @@ def test_planted_mistakes_are_caught(monkeypatch):
     tok.reshape(-1)[:3] = [3.5, 1.25, -3.5]
     codes_no_clip, _, _ = oracle.per_token_quantize(tok, 1.0)
     assert list(codes_no_clip.reshape(-1)[:3]) != [7, 3, -8]
+
+
+# --------------------------------------------------------------------------------------
+# intermediate rounding (x' kept in the input type between the two products)
+# --------------------------------------------------------------------------------------
+
+def test_rounded_intermediate_tie_and_summation_order():
+    """Two hand cases pin the reading. Tie: x' = 1 + 2^-8 is halfway between the bf16
+    neighbours 1 and 1 + 2^-7, so it rounds to the even one, 1 (fp16 holds it exactly).
+    Order: x' = 2^24 + 1 - 2^24 summed in float32 in index order is 0, because 2^24 + 1 rounds
+    to 2^24, while the exact sum is 1. A rounding step dropped, or a sum taken in float64,
+    fails one of them."""
+    P1 = np.ones((1, 1))
+    x = np.array([[[1.0, 2.0 ** -8]]])
+    P2 = np.array([[1.0, 0.0], [1.0, 0.0]])
+    assert oracle.rotate_rounded(x, P1, P2, "bf16")[0, 0, 0] == 1.0
+    assert oracle.rotate_rounded(x, P1, P2, "fp16")[0, 0, 0] == 1.0 + 2.0 ** -8
+    assert oracle.rotate(x, P1, P2)[0, 0, 0] == 1.0 + 2.0 ** -8
+    x = np.array([[[2.0 ** 24, 1.0, -(2.0 ** 24)]]])
+    P2 = np.ones((3, 3))
+    assert np.all(oracle.rotate_rounded(x, P1, P2, "bf16") == 0.0)
+    assert np.all(oracle.rotate(x, P1, P2) == 1.0)
+
+
+def test_round_to_16bit_matches_torch_casts():
+    """The oracle's bf16 rounding (on the float32 bit pattern) and fp16 rounding agree with
+    torch's float32 -> bfloat16 / float16 casts, ties and subnormals included."""
+    rng = _rng(77)
+    v = np.concatenate([
+        (rng.standard_normal(20000) * np.exp(rng.uniform(-30, 30, 20000))).astype(np.float32),
+        np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8), 2.0 ** -130, 0.0, -0.0],
+                 dtype=np.float32)])
+    want_bf = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(oracle.round_to_16bit(v, "bf16"), want_bf)
+    small = v[np.abs(v) < 60000]
+    want_h = torch.from_numpy(small).to(torch.float16).to(torch.float64).numpy()
+    assert np.array_equal(oracle.round_to_16bit(small, "fp16"), want_h)
+
+
+def test_rounded_intermediate_identity_and_skip_reduce_to_exact_path():
+    """With P2 = I every x' sum has one nonzero term, so x' = x exactly and the rounded path
+    equals the exact one; skipping P2 (per-group mode) does too."""
+    rng = _rng(78)
+    x = torch.from_numpy(rng.standard_normal((3, 8, 16))).to(torch.bfloat16).double().numpy()
+    P1 = rng.standard_normal((8, 8))
+    assert np.array_equal(oracle.rotate_rounded(x, P1, np.eye(16)), oracle.rotate(x, P1, np.eye(16)))
+    assert np.array_equal(oracle.rotate_rounded(x, P1, None), oracle.rotate(x, P1, None))
