@@ -109,6 +109,32 @@ def test_bench_host_helpers():
     assert bench.recorded_traffic("nope", "nope", "0") is None
 
 
+def test_bench_reference_arm_json_contract():
+    """`bench.py --impl reference` (the oracle timed on the host cores) prints one JSON line
+    with the keys and types the launcher reads, on the same metric and workload as the
+    CUDA arm. Runs on CPU: the reference arm needs no GPU."""
+    import json
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "0"], capture_output=True, text=True,
+                       timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    for key, typ in [("metric", str), ("value", float), ("unit", str), ("n_gpus", int),
+                     ("steps", int), ("warmup", int), ("ms_per_step", float),
+                     ("higher_is_better", bool), ("scaling", str), ("dtype", str),
+                     ("data", str), ("config", dict), ("cpu_baseline", dict), ("e2e", dict)]:
+        assert isinstance(d[key], typ), (key, d.get(key))
+    assert d["impl"] == "reference" and d["vs_baseline"] is None
+    assert d["value"] > 0 and d["steps"] == 1 and d["n_gpus"] == 1
+    assert d["config"]["workload"] == "mx_case3_32768x128x112"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
 _GLOO_SCRIPT = r"""
 import os, sys
 sys.path.insert(0, {root!r})
