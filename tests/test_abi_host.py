@@ -36,6 +36,40 @@ def test_every_declared_symbol_is_exported(lib):
         assert hasattr(lib, n)
 
 
+_C_PROGRAM = r"""
+#include <stdio.h>
+#include "fq.h"
+int main(void) {
+  fq_handle *h = 0;
+  int bad = 0;
+  /* calls that the library answers from its argument checks, before any CUDA call */
+  bad |= fq_create(0, 4, 16, 16, FQ_BF16) != FQ_ERR_NULLPTR;
+  bad |= fq_create(&h, 0, 16, 16, FQ_BF16) != FQ_ERR_INVALID;
+  bad |= fq_quantize_mx(0, 0, 0, 0, 0.0, 0, 0, 0) != FQ_ERR_NULLPTR;
+  bad |= fq_set_intermediate_rounding(0, 1) != FQ_ERR_NULLPTR;
+  bad |= fq_destroy(0) != FQ_OK;
+  printf("%s\n", fq_status_string(FQ_ERR_INVALID));
+  return bad;
+}
+"""
+
+
+def test_c_program_builds_and_calls_the_abi(lib, tmp_path):
+    """The header is plain C: a C99 program (gcc -pedantic, no CUDA headers) includes it,
+    links against libfq.so and gets the documented status codes back."""
+    from rotation_bit_quantization_token_b200 import _lib
+    src = tmp_path / "abi.c"
+    src.write_text(_C_PROGRAM)
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                    "-L", libdir, "-lfq", f"-Wl,-rpath,{libdir}"], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    assert r.stdout.startswith("FQ_ERR_INVALID")
+
+
 def test_library_is_sm100a_only(lib):
     from rotation_bit_quantization_token_b200 import _lib
     out = subprocess.run(["cuobjdump", "--list-elf", _lib.LIB_PATH], capture_output=True, text=True)
