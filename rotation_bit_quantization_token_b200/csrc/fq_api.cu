@@ -40,19 +40,6 @@ fq_status cuda_fail(cudaError_t e) {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// Per-group rule from dstTypeMax (page: per-group mode, cases 1-3). Returns false for a
-// value outside {0} U [6, 12] (parameter table: "0.0 disables, 6.0~12.0 customizes").
-bool mx_rule_from(double d, fq::MxRule* r) {
-  if (!(d == 0.0 || (d >= 6.0 && d <= 12.0))) return false;
-  if (d == 0.0) r->mode = fq::kMxFloor;
-  else if (d == 6.0) r->mode = fq::kMxMantissa6;
-  else if (d == 7.0) r->mode = fq::kMxMantissa7;
-  else r->mode = fq::kMxRatio;
-  r->dst_max = float(d);
-  r->inv_dst = d > 0.0 ? float(1.0 / d) : 0.0f;
-  return true;
-}
-
 // The tensor-core kernel moves x with TMA, P1 / P2 with 16-byte loads and the outputs
 // with bulk copies, so all of them must be 16-byte aligned.
 bool use_tc(const fq_handle* h, const void* x, const void* P1, const void* P2, const void* out,
@@ -103,6 +90,17 @@ fq_status launch(fq_handle* h, int mode, const void* x, const void* P1, const vo
 }  // namespace
 
 void fq::record_cuda_error(int e) { g_last_cuda_error = e; }
+
+bool fq::mx_rule_from(double d, fq::MxRule* r) {
+  if (!(d == 0.0 || (d >= 6.0 && d <= 12.0))) return false;
+  if (d == 0.0) r->mode = fq::kMxFloor;
+  else if (d == 6.0) r->mode = fq::kMxMantissa6;
+  else if (d == 7.0) r->mode = fq::kMxMantissa7;
+  else r->mode = fq::kMxRatio;
+  r->dst_max = float(d);
+  r->inv_dst = d > 0.0 ? float(1.0 / d) : 0.0f;
+  return true;
+}
 
 extern "C" {
 
@@ -174,7 +172,7 @@ fq_status fq_quantize_mx(fq_handle* h, const void* x, const void* P1, const void
       scale_e8m0 == nullptr)
     return FQ_ERR_NULLPTR;
   fq::MxRule rule;
-  if (!mx_rule_from(dstTypeMax, &rule)) return FQ_ERR_INVALID;
+  if (!fq::mx_rule_from(dstTypeMax, &rule)) return FQ_ERR_INVALID;
   if (h->N % 2 != 0) return FQ_ERR_INVALID;  // page: FLOAT4_E2M1 needs N even
   if (!aligned(x, 2) || !aligned(P1, 2) || (P2 != nullptr && !aligned(P2, 2)))
     return FQ_ERR_INVALID;

@@ -52,6 +52,11 @@ struct TcParams {
 
 bool tc_supported(int64_t K, int M, int N);
 
+// Per-group rule from dstTypeMax (page: per-group mode, cases 1-3). Returns false for a
+// value outside {0} U [6, 12] (parameter table: "0.0 disables, 6.0~12.0 customizes").
+// The one decoding used by every per-group entry point.
+bool mx_rule_from(double dst_type_max, MxRule* rule);
+
 // Keeps a CUDA error code for fq_last_cuda_error() (thread-local).
 void record_cuda_error(int e);
 cudaError_t launch_tc(const TcParams& p, bool fp16_in, int num_sms, cudaStream_t stream);

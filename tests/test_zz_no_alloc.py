@@ -5,10 +5,14 @@ allocator or a fixed budget, or a cudaMalloc would synchronize a latency-critica
 This entry point keeps its only scratch, a status word, in a static device array of the
 library. The test calls it through the C ABI twice in a row and checks that it writes the
 same codes and scales as the allocating entry point (fq_quantize_mx through a handle),
-which the parity tests hold to the oracle. It sits in a file of its own, collected last.
+which the parity tests hold to the oracle, and that fq_static_device_status reads the word
+back as 0. A second test makes one launch's bounded wait run out (the process-wide
+one-shot fq_static_debug_arm_stall; no fault, a 50 ms limit) and checks that the reader
+reports it and that the next call is correct again. The file is collected last.
 """
 
 import ctypes
+import time
 
 import pytest
 import torch
@@ -47,6 +51,43 @@ def test_static_scratch_matches_allocating_entry_point(w):
         torch.cuda.synchronize()
         assert torch.equal(out, ref_out)
         assert torch.equal(sc, ref_sc)
+        assert _static_status(lib) == (_lib.FQ_OK, 0)
+
+
+def _static_status(lib):
+    v = ctypes.c_uint32(0xFFFFFFFF)
+    st = lib.fq_static_device_status(ctypes.byref(v))
+    return st, int(v.value)
+
+
+def test_static_path_reports_an_expired_wait():
+    lib = _lib.load()
+    dev = torch.device("cuda", 0)
+    w = WORKLOADS["mx_case3_32768x128x112"].with_tokens(300)
+    x, P1, P2 = (t.to(dev) for t in make_inputs(w, seed=7))
+    ref_out, ref_sc = FlatQuant(w.K, w.M, w.N).quantize_mx(x, P1, P2, w.dst_type_max)
+    out = torch.empty_like(ref_out)
+    sc = torch.empty_like(ref_sc)
+    torch.cuda.synchronize()
+    assert _static_status(lib) == (_lib.FQ_OK, 0)
+    assert lib.fq_static_debug_arm_stall(0.05) == _lib.FQ_OK
+    t0 = time.monotonic()
+    assert _call_static(lib, x, P1, P2, w.dst_type_max, out, sc) == _lib.FQ_OK
+    torch.cuda.synchronize()
+    elapsed = time.monotonic() - t0
+    st, v = _static_status(lib)
+    assert st == _lib.FQ_ERR_DEVICE_TIMEOUT and v != 0, (st, v)
+    assert v & 2, f"stage A's wait for the x tile is not among the expired waits ({v:#x})"
+    assert elapsed < 2.0
+    assert _static_status(lib) == (_lib.FQ_OK, 0)  # the read cleared it
+    # the hook is one-shot: the next call runs normally
+    assert _call_static(lib, x, P1, P2, w.dst_type_max, out, sc) == _lib.FQ_OK
+    torch.cuda.synchronize()
+    assert _static_status(lib) == (_lib.FQ_OK, 0)
+    assert torch.equal(out, ref_out) and torch.equal(sc, ref_sc)
+    for bad in (0.0, -1.0, 11.0, float("nan")):
+        assert lib.fq_static_debug_arm_stall(bad) == _lib.FQ_ERR_INVALID
+    assert lib.fq_static_device_status(None) == _lib.FQ_ERR_NULLPTR
 
 
 def test_static_entry_point_rejects_bad_arguments():
