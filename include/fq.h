@@ -32,6 +32,9 @@
  *     shape / range / type rule the page lists. A launch failure is FQ_ERR_CUDA; the
  *     CUDA error is kept and returned by fq_last_cuda_error(). Execution faults surface
  *     on the stream as usual.
+ *   - Inputs are finite numbers. For a group whose float32 absmax is not finite, the
+ *     ratio rule (case 3) gives the byte 0xFF (the rule applied to an infinite S) and the
+ *     codes of that group are unspecified; a NaN in x is outside the contract.
  *   - Pointers need the alignment of their element type; 16-byte aligned x, out and
  *     scale pointers (and M*N a multiple of 32) let the tensor-core kernel run, other
  *     cases take the general kernel.
@@ -124,26 +127,48 @@ FQ_API fq_status fq_quantize_mx(fq_handle *h, const void *x, const void *P1, con
  * takes the shape and dtype directly (no handle), allocates nothing and frees nothing:
  * no cudaMalloc, cudaFree or allocating library routine runs in it.
  *
- * Its only scratch is one 32-bit status word (the word a kernel sets when one of its
- * bounded waits gives up) inside a 256-byte static device array of the library. That
- * array is loaded with the library's device code and held on every GPU that uses it
- * until the process exits. Each call clears the word with cudaMemsetAsync on `stream`
- * before the launch; the array otherwise keeps what the last call left. All calls in the
- * process share the array, so calls that overlap on the GPU race on that word.
+ * Its only scratch is one 32-bit status word (the word the tensor-core kernel sets when
+ * one of its bounded waits gives up) inside a 256-byte static device array of the
+ * library. That array is loaded with the library's device code and held on every GPU that
+ * uses it until the process exits. A call that launches the tensor-core kernel clears the
+ * word with cudaMemsetAsync on `stream` before the launch; the array otherwise keeps what
+ * the last call left. All calls in the process share the array, so calls that overlap on
+ * the GPU race on that word. fq_static_device_status reads the word back: a wait that
+ * gave up leaves the outputs of that call undefined, and this reader is the only way to
+ * learn of it on this path.
  *
- * The first call on a device looks up the array's device address (cudaGetSymbolAddress,
- * with that device current) and caches it; make that first call before any stream
- * capture. Arguments, layouts and errors are those of fq_quantize_mx plus the plan-phase
- * checks of fq_create (K in [1, 262144], M, N in [1, 256], dtype): FQ_ERR_NULLPTR,
- * FQ_ERR_INVALID (including a call whose scratch would exceed the static array, which no
- * allowed shape does), FQ_ERR_UNSUPPORTED, FQ_ERR_CUDA. */
+ * Every call looks up the array's device address in the current context
+ * (cudaGetSymbolAddress, a host-side query). The first call in a process or context may
+ * also load the library's device code, so make it before any stream capture. Arguments,
+ * layouts and errors are those of fq_quantize_mx plus the plan-phase checks of fq_create
+ * (K in [1, 262144], M, N in [1, 256], dtype): FQ_ERR_NULLPTR, FQ_ERR_INVALID (including
+ * a call whose scratch would exceed the static array, which no allowed shape does),
+ * FQ_ERR_UNSUPPORTED, FQ_ERR_CUDA. */
 FQ_API fq_status fq_quantize_mx_static(int64_t K, int64_t M, int64_t N, fq_dtype dtype,
                                        const void *x, const void *P1, const void *P2,
                                        double dstTypeMax, void *out_fp4, uint8_t *scale_e8m0,
                                        struct CUstream_st *stream);
 
-/* Test hook: writes x'' = P1 . (x . P2) as float32 [K, M, N] (P2 may be NULL), computed
- * the way the selected kernel computes it before quantization. */
+/* Reads and clears the status word of fq_quantize_mx_static on the current device (the
+ * paper has no counterpart). *status = 0 when no launch of that entry point gave up a
+ * bounded wait since the word was last cleared, else the code of the wait (and the call
+ * returns FQ_ERR_DEVICE_TIMEOUT). Synchronizes with the device (a blocking copy) and
+ * allocates nothing. Returns FQ_ERR_NULLPTR for a NULL status, FQ_ERR_CUDA if the copy
+ * fails. */
+FQ_API fq_status fq_static_device_status(uint32_t *status);
+
+/* Test hook for the failure path of fq_quantize_mx_static (the paper has no counterpart):
+ * process-wide and one-shot, like fq_debug_arm_stall for a handle. The next call of
+ * fq_quantize_mx_static in this process that takes the tensor-core kernel issues no x loads
+ * and gives every bounded wait a limit of wait_limit_s seconds (0 < wait_limit_s <= 10), so
+ * its first stage-A wait runs out, the kernel sets the status word and returns; the outputs
+ * of that call are undefined. Returns FQ_ERR_INVALID for a limit out of range. */
+FQ_API fq_status fq_static_debug_arm_stall(double wait_limit_s);
+
+/* Test hook: writes x'' = P1 . (x . P2) ("How it works", the two-level matmul) as float32
+ * [K, M, N] (P2 may be NULL), computed the way the selected kernel computes it before
+ * quantization. The page exposes no such output; it lets tests compare the rotation alone.
+ * Errors: FQ_ERR_NULLPTR (h, x, P1, x2), FQ_ERR_INVALID (misaligned pointer), FQ_ERR_CUDA. */
 FQ_API fq_status fq_debug_rotate(fq_handle *h, const void *x, const void *P1, const void *P2,
                           float *x2, struct CUstream_st *stream);
 
@@ -186,7 +211,9 @@ FQ_API fq_status fq_device_status(fq_handle *h, uint32_t *status);
 /* The CUDA error code kept by the last call that returned FQ_ERR_CUDA in this thread. */
 FQ_API int fq_last_cuda_error(void);
 
-/* Static description of a status code. */
+/* Static description of a status code (the codes follow the page's "Error code quick
+ * reference"; the page has no such function). Never NULL; unknown codes give
+ * "unknown fq_status". */
 FQ_API const char *fq_status_string(fq_status s);
 
 #ifdef __cplusplus

@@ -31,6 +31,12 @@ __device__ __forceinline__ float pow2_from_e8m0_inverse(uint32_t b) {
   return __uint_as_float((254u - b) << 23);
 }
 
+// The same for every byte the ratio rule can give: 254 is 2^-127 (a subnormal), and 255,
+// the byte of a non-finite S, gets 0 (1 / infinity), so no byte wraps the exponent field.
+__device__ __forceinline__ float pow2_from_e8m0_inverse_any(uint32_t b) {
+  return b <= 253u ? pow2_from_e8m0_inverse(b) : (b == 254u ? __uint_as_float(0x00400000u) : 0.0f);
+}
+
 // Shared exponent of one group from its float32 absolute maximum.
 //  case 1 (0.0):     e = floor(log2 amax) - 2, clamped to [-127, 127]
 //  case 2 (6.0/7.0): e = floor(log2 amax) - 2 + [leading one/two fraction bits set and
@@ -42,16 +48,16 @@ template <bool kExactDiv = true>
 __device__ __forceinline__ MxScale mx_scale(float amax, MxRule rule) {
   MxScale s;
   if (rule.mode == kMxRatio) {
-    // S = amax / dstTypeMax in float32. The tensor-core kernel multiplies by the
-    // float32 reciprocal instead (kExactDiv = false): the product is within one ulp of
-    // the quotient, which moves the byte only when amax / dstTypeMax is a power of two.
+    // S = amax / dstTypeMax in float32, rounded to nearest (both kernels). kExactDiv =
+    // false would multiply by the float32 reciprocal instead: within one ulp of the
+    // quotient, which can move the byte when amax / dstTypeMax is a power of two.
     const float S = kExactDiv ? __fdiv_rn(amax, rule.dst_max) : amax * rule.inv_dst;
     const uint32_t bits = __float_as_uint(S);
     uint32_t E = (bits >> 23) & 0xFFu;
     const uint32_t mant = bits & 0x7FFFFFu;
     if (E >= 1u && E < 254u && mant != 0u) E += 1u;
     s.byte = E;
-    s.R = pow2_from_e8m0_inverse(E);
+    s.R = pow2_from_e8m0_inverse_any(E);  // E is 255 only for a non-finite S
     return s;
   }
   const uint32_t bits = __float_as_uint(amax);

@@ -870,7 +870,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
           if constexpr ((N % 32) == 0) {
 #pragma unroll
             for (int gi = 0; gi < NS / 2; ++gi) {
-              const MxScale ms = mx_scale<false>(fmaxf(smax[2 * gi], smax[2 * gi + 1]) * fcrow, p.rule);
+              const MxScale ms = mx_scale<true>(fmaxf(smax[2 * gi], smax[2 * gi + 1]) * fcrow, p.rule);
               const float F = exp2i(127 - int(ms.byte) + crow);
               Fseg[2 * gi] = F;
               Fseg[2 * gi + 1] = F;
@@ -883,14 +883,14 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
             const bool odd = (row & 1) != 0;
             const float part = (odd ? smax[0] : smax[NS - 1]) * fcrow;
             const float other = __shfl_xor_sync(0xffffffffu, part, 1);
-            const MxScale mst = mx_scale<false>(fmaxf(part, other), p.rule);
+            const MxScale mst = mx_scale<true>(fmaxf(part, other), p.rule);
             const float Fst = exp2i(127 - int(mst.byte) + crow);
             const int pair_base = (row >> 1) * (N / 16);
             float Ff[GF];
 #pragma unroll
             for (int gi = 0; gi < GF; ++gi) {
               const float a = odd ? fmaxf(smax[2 * gi + 1], smax[2 * gi + 2]) : fmaxf(smax[2 * gi], smax[2 * gi + 1]);
-              const MxScale ms = mx_scale<false>(a * fcrow, p.rule);
+              const MxScale ms = mx_scale<true>(a * fcrow, p.rule);
               Ff[gi] = exp2i(127 - int(ms.byte) + crow);
               s_scale[pair_base + (odd ? GF + 1 : 0) + gi] = uint8_t(ms.byte);
             }
