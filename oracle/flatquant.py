@@ -101,25 +101,95 @@ def round_to_16bit(v, dtype):
     return bits.astype(np.uint32).view(np.float32).astype(np.float64)
 
 
+# significant bits, smallest normal exponent and largest finite value of the 16-bit types
+_FMT16 = {"bf16": (8, -126, (2.0 - 2.0 ** -7) * 2.0 ** 127),
+          "fp16": (11, -14, 65504.0)}
+
+
+def _quantum16(a, dtype):
+    """Spacing of the 16-bit type's values around magnitudes a (float64 array, a >= 0):
+    2^(e - (p - 1)) in the binade [2^e, 2^(e+1)), the subnormal spacing below 2^emin."""
+    p, emin, _ = _FMT16[dtype]
+    e = _floor_log2(np.where(a > 0, a, 1.0))
+    e = np.maximum(e, emin)
+    return np.ldexp(1.0, e - (p - 1))
+
+
+def round_f64_to_16bit(v, dtype):
+    """float64 values rounded directly (no float32 step) to the nearest "bf16" / "fp16"
+    value, ties to the even significand; magnitudes at or beyond the midpoint between the
+    largest finite value and the next power of two become infinite. Returned as float64.
+    The division by the spacing is exact (a power of two) and numpy's rint rounds half to
+    even."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    q = _quantum16(a, dtype)
+    r = np.rint(a / q) * q
+    _, _, top = _FMT16[dtype]
+    r = np.where(r > top, np.inf, r)
+    return np.copysign(r, v)
+
+
+def _round_fraction_16bit(fr, dtype):
+    """Exact rational fr rounded to the 16-bit type (nearest, ties to even): the
+    definition itself, in integer arithmetic."""
+    from fractions import Fraction
+    if fr == 0:
+        return 0.0
+    p, emin, top = _FMT16[dtype]
+    a = abs(fr)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1                                  # now 2^e <= a < 2^(e+1)
+    q = Fraction(2) ** (max(e, emin) - (p - 1))
+    k = a / q
+    n = k.numerator // k.denominator            # floor
+    rem = k - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    r = float(n * q) if n * q <= Fraction(top) else float("inf")
+    return r if fr > 0 else -r
+
+
+def round16_of_exact_product(x, P2, dtype):
+    """x' = x . P2 with every element rounded once, from its exact value, to the 16-bit
+    type (nearest, ties to even). x [..., M, N] and P2 [N, N] hold 16-bit values, so each
+    product is exact in float64; the float64 matmul is within N * 2^-52 * (|x| . |P2|) of
+    the exact sum, so its rounding is the rounding of the exact sum unless a rounding
+    midpoint lies inside that bound. Those elements (rare) are summed exactly as rationals
+    and rounded by definition."""
+    from fractions import Fraction
+    x = np.asarray(x, dtype=np.float64)
+    P2 = np.asarray(P2, dtype=np.float64)
+    N = P2.shape[0]
+    v = np.matmul(x, P2)
+    bound = (N * 2.0 ** -52) * 1.01 * np.matmul(np.abs(x), np.abs(P2))
+    a = np.abs(v)
+    q = _quantum16(a, dtype)
+    mid = (np.floor(a / q) + 0.5) * q
+    near = np.abs(a - mid) <= bound
+    out = round_f64_to_16bit(v, dtype)
+    for idx in zip(*np.nonzero(near)):
+        row = x[idx[:-1]]
+        col = P2[:, idx[-1]]
+        exact = sum(Fraction(float(row[j])) * Fraction(float(col[j])) for j in range(N))
+        out[idx] = _round_fraction_16bit(exact, dtype)
+    return out
+
+
 def rotate_rounded(x, P1, P2, dtype="bf16"):
     """Two-level small matmul with x' kept in the input type between the products: the
     intermediate-rounding reading of "How it works", whose formulas leave the precision of
-    x' open. Each x'[m, n] is the sum over j = 0, 1, ..., N-1, in that order, of
-    x[m, j] * P2[j, n] in float32: every partial sum is rounded to float32, and the
-    product of two 16-bit inputs is exact in float32. The sum is then rounded to the input
-    type (nearest, ties to even), and x'' = P1 . x' is formed in float64.
-    P2 None or empty skips the right multiply (x' = x, already in the input type)."""
+    x' open. x' = x . P2 is formed exactly and each element is rounded once to the input
+    type (nearest, ties to even); x'' = P1 . x' is then formed in float64 from the rounded
+    values. No summation order is assumed for x'. P2 None or empty skips the right
+    multiply (x' = x, already in the input type)."""
     x = np.asarray(x, dtype=np.float64)
     P1 = np.asarray(P1, dtype=np.float64)
     if P2 is None or np.size(P2) == 0:
         x1 = x
     else:
-        x32 = x.astype(np.float32)
-        P2_32 = np.asarray(P2, dtype=np.float32)
-        acc = np.zeros(x.shape, dtype=np.float32)
-        for j in range(x.shape[-1]):
-            acc = (acc + x32[..., j:j + 1] * P2_32[j]).astype(np.float32)
-        x1 = round_to_16bit(acc, dtype)
+        x1 = round16_of_exact_product(x, P2, dtype)
     return np.matmul(P1, x1)
 
 

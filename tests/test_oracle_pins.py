@@ -389,12 +389,13 @@ def test_planted_mistakes_are_caught(monkeypatch):
 # intermediate rounding (x' kept in the input type between the two products)
 # --------------------------------------------------------------------------------------
 
-def test_rounded_intermediate_tie_and_summation_order():
-    """Two hand cases pin the reading. Tie: x' = 1 + 2^-8 is halfway between the bf16
-    neighbours 1 and 1 + 2^-7, so it rounds to the even one, 1 (fp16 holds it exactly).
-    Order: x' = 2^24 + 1 - 2^24 summed in float32 in index order is 0, because 2^24 + 1 rounds
-    to 2^24, while the exact sum is 1. A rounding step dropped, or a sum taken in float64,
-    fails one of them."""
+def test_rounded_intermediate_tie_and_exact_sum():
+    """Hand cases pin the reading x' = round16(exact x . P2). Tie: x' = 1 + 2^-8 is halfway
+    between the bf16 neighbours 1 and 1 + 2^-7, so it rounds to the even one, 1 (fp16 holds
+    it exactly). Exactness: 2^24 + 1 - 2^24 is 1 (a float32 running sum in index order would
+    give 0). Just above the tie: 1 + 2^-8 + 2^-60 rounds up to 1 + 2^-7, although its float64
+    sum is the tie itself (this takes the oracle's exact-rational branch). A rounding step
+    dropped, a float32 or float64 sum used as if exact, or a wrong tie rule fails one."""
     P1 = np.ones((1, 1))
     x = np.array([[[1.0, 2.0 ** -8]]])
     P2 = np.array([[1.0, 0.0], [1.0, 0.0]])
@@ -403,8 +404,77 @@ def test_rounded_intermediate_tie_and_summation_order():
     assert oracle.rotate(x, P1, P2)[0, 0, 0] == 1.0 + 2.0 ** -8
     x = np.array([[[2.0 ** 24, 1.0, -(2.0 ** 24)]]])
     P2 = np.ones((3, 3))
-    assert np.all(oracle.rotate_rounded(x, P1, P2, "bf16") == 0.0)
-    assert np.all(oracle.rotate(x, P1, P2) == 1.0)
+    assert np.all(oracle.rotate_rounded(x, P1, P2, "bf16") == 1.0)
+    x = np.array([[[1.0, 2.0 ** -8, 2.0 ** -60]]])
+    P2 = np.zeros((3, 3))
+    P2[:, 0] = 1.0
+    assert oracle.rotate_rounded(x, P1, P2, "bf16")[0, 0, 0] == 1.0 + 2.0 ** -7
+    assert oracle.rotate_rounded(x, P1, P2, "fp16")[0, 0, 0] == 1.0 + 2.0 ** -8
+    x = np.array([[[-1.0, -(2.0 ** -8), -(2.0 ** -60)]]])
+    assert oracle.rotate_rounded(x, P1, P2, "bf16")[0, 0, 0] == -(1.0 + 2.0 ** -7)
+
+
+def _int_round_half_even(num, shift):
+    """num / 2^shift (shift >= 0) rounded to an integer, ties to even, in integers."""
+    if shift == 0:
+        return num
+    q, r = divmod(num, 1 << shift)
+    half = 1 << (shift - 1)
+    if r > half or (r == half and q % 2 == 1):
+        q += 1
+    return q
+
+
+def test_rounded_intermediate_on_integer_grid_matches_integer_arithmetic():
+    """x on the grid k / 8 and P2 on the grid j / 16 (|k|, |j| <= 15): every x' element is an
+    integer multiple of 2^-7, computed here with Python integers. Rounded to 8 significant
+    bits (bf16) or 11 (fp16) with an integer ties-to-even rule, it must equal the oracle's x'
+    (read back through P1 = I). Ties occur on this grid, so a wrong tie rule, a truncation or
+    a transposed P2 fails."""
+    rng = _rng(79)
+    K, M, N = 3, 8, 24
+    xi = rng.integers(-15, 16, size=(K, M, N))
+    pi = rng.integers(-15, 16, size=(N, N))
+    x = xi / 8.0
+    P2 = pi / 16.0
+    ties = 0
+    for dtype, p in (("bf16", 8), ("fp16", 11)):
+        got = oracle.rotate_rounded(x, np.eye(M), P2, dtype)
+        for k in range(K):
+            for m in range(M):
+                for n in range(N):
+                    s = int(sum(int(xi[k, m, j]) * int(pi[j, n]) for j in range(N)))  # x' * 2^7
+                    a = abs(s)
+                    if a == 0:
+                        want = 0.0
+                    else:
+                        shift = max(a.bit_length() - p, 0)
+                        r = _int_round_half_even(a, shift)
+                        want = float(r) * 2.0 ** (shift - 7)
+                        if shift > 0 and a % (1 << shift) == 1 << (shift - 1):
+                            ties += 1
+                    want = -want if s < 0 else want
+                    assert got[k, m, n] == want, (dtype, k, m, n, s)
+    assert ties > 0
+
+
+def test_round_f64_to_16bit_ties_subnormals_overflow():
+    """Direct float64 -> 16-bit rounding: agrees with torch's casts on float32 values (ties
+    and subnormals included); a value just above a tie, which a float32 step would turn into
+    the tie, rounds up; fp16 overflows to inf at 65520 and keeps 65504 below it; half the
+    smallest fp16 subnormal rounds to 0 (even), three quarters of it to 2^-24."""
+    rng = _rng(80)
+    v = np.concatenate([
+        (rng.standard_normal(20000) * np.exp(rng.uniform(-30, 30, 20000))).astype(np.float32),
+        np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8), 2.0 ** -130, 0.0], dtype=np.float32)])
+    want_bf = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(fq.round_f64_to_16bit(v.astype(np.float64), "bf16"), want_bf)
+    small = v[np.abs(v) < 60000]
+    want_h = torch.from_numpy(small).to(torch.float16).to(torch.float64).numpy()
+    assert np.array_equal(fq.round_f64_to_16bit(small.astype(np.float64), "fp16"), want_h)
+    assert fq.round_f64_to_16bit(np.array([1 + 2 ** -8 + 2 ** -40]), "bf16")[0] == 1 + 2 ** -7
+    h = fq.round_f64_to_16bit(np.array([65519.99, 65520.0, 2.0 ** -25, 0.75 * 2.0 ** -24]), "fp16")
+    assert h[0] == 65504.0 and np.isinf(h[1]) and h[2] == 0.0 and h[3] == 2.0 ** -24
 
 
 def test_round_to_16bit_matches_torch_casts():
