@@ -62,15 +62,23 @@ def group_exempt(amax, D):
     return _near_pow2(amax / D)
 
 
-def compare_per_token(out_bytes, qs, ref_codes, ref_qs, ref_v):
-    """out_bytes: uint8 [K, M*N/2] from the GPU; ref_* from oracle.per_token_quantize."""
+def compare_per_token(out_bytes, qs, ref_codes, ref_qs, ref_v, elem_taint=None, token_taint=None):
+    """out_bytes: uint8 [K, M*N/2] from the GPU; ref_* from oracle.per_token_quantize.
+    elem_taint [K, M*N] / token_taint [K] (optional) mark elements and whole tokens whose
+    reference value is not decided by the inputs alone (see intermediate_rounding_taint):
+    tainted elements are exempt, tainted tokens are skipped."""
     K = ref_codes.shape[0]
-    got = unpack_nibbles(np.asarray(out_bytes).reshape(K, -1)).astype(np.int64)
+    keep = np.ones(K, dtype=bool) if token_taint is None else ~np.asarray(token_taint)
+    got = unpack_nibbles(np.asarray(out_bytes).reshape(K, -1)).astype(np.int64)[keep]
     got = np.where(got >= 8, got - 16, got)
-    want = ref_codes.reshape(K, -1).astype(np.int64)
-    v = ref_v.reshape(K, -1)
+    want = ref_codes.reshape(K, -1).astype(np.int64)[keep]
+    v = ref_v.reshape(K, -1)[keep]
     diff = got != want
     exempt = int4_exempt(v)
+    if elem_taint is not None:
+        exempt = exempt | np.asarray(elem_taint).reshape(K, -1)[keep]
+    qs = np.asarray(qs)[keep]
+    ref_qs = np.asarray(ref_qs)[keep]
     stats = {"elements": int(want.size), "mismatch": int(diff.sum()),
              "exempt_mismatch": int((diff & exempt).sum())}
     bad = diff & ~exempt
@@ -93,9 +101,11 @@ def _e2m1_step(a_codes, b_codes):
     return np.abs(pos(a_codes) - pos(b_codes))
 
 
-def compare_mx(out_bytes, scales, ref_info, D):
+def compare_mx(out_bytes, scales, ref_info, D, elem_taint=None):
     """out_bytes uint8 [K, M*N/2], scales uint8 [K, S, 2] from the GPU; ref_info from
-    oracle.flat_quant_mx."""
+    oracle.flat_quant_mx. elem_taint [K, M*N] (optional) marks elements whose reference
+    value is not decided by the inputs alone: every group holding one is exempt, its
+    byte and its codes (see intermediate_rounding_taint)."""
     ref_codes = ref_info["codes"]
     K, L = ref_codes.shape
     G = ref_info["group_bytes"].shape[1]
@@ -107,6 +117,10 @@ def compare_mx(out_bytes, scales, ref_info, D):
         assert np.all(got_b[:, G:] == 0), "pad scale byte is not 0x00"
     got_b = got_b[:, :G].astype(np.int64)
     gex = group_exempt(ref_info["amax"], D)
+    if elem_taint is not None:
+        t = np.zeros((K, G * 32), dtype=bool)
+        t[:, :L] = np.asarray(elem_taint).reshape(K, -1)
+        gex = gex | t.reshape(K, G, 32).any(axis=-1)
     bdiff = got_b != want_b.astype(np.int64)
     assert not (bdiff & ~gex).any(), \
         f"non-exempt E8M0 mismatches: {int((bdiff & ~gex).sum())}"
@@ -127,15 +141,67 @@ def compare_mx(out_bytes, scales, ref_info, D):
     return stats
 
 
-def rotate_close(x2_gpu, x2_ref):
-    """x'' within 2e-3 relative: |d| <= 2e-3 * max(|ref|, 1e-3 * amax_token). Returns the
-    largest error divided by the token's rms (a finer figure that is reported)."""
+def rotate_close(x2_gpu, x2_ref, extra=None):
+    """x'' within 2e-3 relative: |d| <= 2e-3 * max(|ref|, 1e-3 * amax_token) (+ extra, an
+    optional per-element allowance). Returns the largest error divided by the token's rms
+    (a finer figure that is reported)."""
     K = x2_ref.shape[0]
     g = np.asarray(x2_gpu, dtype=np.float64).reshape(K, -1)
     r = np.asarray(x2_ref, dtype=np.float64).reshape(K, -1)
     amax = np.abs(r).max(axis=1, keepdims=True)
     tol = 2e-3 * np.maximum(np.abs(r), 1e-3 * amax)
+    if extra is not None:
+        tol = tol + np.asarray(extra, dtype=np.float64).reshape(K, -1)
     d = np.abs(g - r)
     assert np.all(d <= tol), f"x'' outside tolerance: worst {float((d / np.maximum(tol, 1e-300)).max())}"
     rms = np.sqrt((r * r).mean(axis=1, keepdims=True))
     return float((d / np.maximum(rms, 1e-300)).max())
+
+
+# --------------------------------------------------------------------------------------
+# intermediate-rounding mode: which reference values the inputs do not decide
+# --------------------------------------------------------------------------------------
+
+_P16 = {"bf16": (8, -126), "fp16": (11, -14)}
+
+
+def _spacing16(a, dtype):
+    """Spacing of 16-bit values around magnitudes a (the quantum of their binade)."""
+    p, emin = _P16[dtype]
+    a = np.asarray(a, dtype=np.float64)
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))
+    e = np.maximum(ex.astype(np.int64) - 1, emin)
+    return np.ldexp(1.0, e - (p - 1))
+
+
+def intermediate_rounding_taint(x, P1, P2, dtype):
+    """In the intermediate-rounding mode x' = round16(x . P2). A kernel forms x . P2 in
+    float32 in some order, so its sum can lie anywhere within N * 2^-24 * sum_j |x_j P2_jn|
+    of the exact one; where a 16-bit rounding midpoint lies inside that bound, the kernel
+    may round x' to the other neighbour, one 16-bit spacing away. Returns (dev [K, M, N]:
+    the largest change of each x'' element that such roundings can cause, sum over m of
+    |P1[r, m]| * spacing(x'[m, n]) for the x'[m, n] so marked; x1_taint [K, M, N]: the x'
+    elements marked). Elements of x'' with dev > 0 are not decided by the inputs."""
+    x = np.asarray(x, dtype=np.float64)
+    P2 = np.asarray(P2, dtype=np.float64)
+    N = P2.shape[0]
+    v = np.matmul(x, P2)
+    bound = N * 2.0 ** -24 * 1.01 * np.matmul(np.abs(x), np.abs(P2))
+    a = np.abs(v)
+    q = _spacing16(a, dtype)
+    mid = (np.floor(a / q) + 0.5) * q
+    lower_mid = (np.floor(a / q) - 0.5) * q  # the midpoint below, for values just above one
+    taint = (np.abs(a - mid) <= bound) | (np.abs(a - lower_mid) <= bound)
+    step = np.where(taint, 2.0 * q, 0.0)   # the binade may change at a power of two
+    dev = np.matmul(np.abs(np.asarray(P1, dtype=np.float64)), step)
+    return dev, taint
+
+
+def token_taint_from(dev, x2_ref):
+    """Tokens whose absolute maximum the tainted elements can change (their per-token
+    scale, and so every code, is then not decided by the inputs)."""
+    K = x2_ref.shape[0]
+    d = np.asarray(dev).reshape(K, -1)
+    r = np.abs(np.asarray(x2_ref, dtype=np.float64)).reshape(K, -1)
+    amax = r.max(axis=1)
+    return (d > 0).any(axis=1) & ((r + d).max(axis=1) >= amax - d.max(axis=1))

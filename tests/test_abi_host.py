@@ -70,12 +70,14 @@ def test_c_program_builds_and_calls_the_abi(lib, tmp_path):
     assert r.stdout.startswith("FQ_ERR_INVALID")
 
 
-def test_library_is_sm100a_only(lib):
-    from rotation_bit_quantization_token_b200 import _lib
-    out = subprocess.run(["cuobjdump", "--list-elf", _lib.LIB_PATH], capture_output=True, text=True)
-    if out.returncode != 0:
-        pytest.skip("cuobjdump unavailable")
-    assert "sm_100a" in out.stdout
+def test_library_is_built_for_sm100a_only():
+    """The build compiles every source for sm_100a alone: one -gencode pair, compute_100a
+    to sm_100a, for the objects and for the link (no PTX for other targets)."""
+    from rotation_bit_quantization_token_b200 import build
+    flags = build.NVCC_FLAGS
+    pairs = [flags[i + 1] for i, f in enumerate(flags) if f == "-gencode"]
+    assert pairs == ["arch=compute_100a,code=sm_100a"]
+    assert not any(f.startswith("-arch") or f.startswith("--gpu-architecture") for f in flags)
 
 
 def test_plan_validation_without_device(lib):
@@ -167,6 +169,25 @@ def test_bench_reference_arm_json_contract():
     assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
+    # it reports what it timed: the per-step time of its sample, not an extrapolation to
+    # the whole workload, so the steps fit in the run
+    n = d["config"]["tokens_per_step_sample"]
+    assert 1 <= n <= d["config"]["K"]
+    assert abs(d["value"] - n / (d["ms_per_step"] / 1e3)) <= 1e-6 * d["value"]
+    assert d["cpu_baseline"]["nproc"] >= d["cpu_baseline"]["usable_cores"] >= 1
+
+
+def test_bench_buffer_copies_exceed_l2():
+    """Workloads smaller than twice the L2 cycle through enough copies to exceed it."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from rotation_bit_quantization_token_b200.workloads import WORKLOADS
+    assert bench.buffer_copies(WORKLOADS["mx_case3_32768x128x112"].bytes_per_token() * 32768) == 1
+    for name in WORKLOADS:
+        b = WORKLOADS[name].bytes_per_token() * WORKLOADS[name].K
+        c = bench.buffer_copies(b)
+        assert c * b > 2 * bench.L2_BYTES
+        assert c == 1 or (c - 1) * b <= 2 * bench.L2_BYTES + b
 
 
 _GLOO_SCRIPT = r"""
