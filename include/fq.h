@@ -117,6 +117,34 @@ FQ_API fq_status fq_quantize_mx(fq_handle *h, const void *x, const void *P1, con
                          double dstTypeMax, void *out_fp4, uint8_t *scale_e8m0,
                          struct CUstream_st *stream);
 
+/* Consumer of two per-group outputs: the FP4 x FP4 contraction with E8M0 block scales.
+ * The page ("per-token mode"; its summary on FP4 E2M1 compression of weights and
+ * activations) says the quantized data and scales are emitted for later dequantization
+ * and low-precision compute; this is that compute for activations A and weights W that
+ * both come out of fq_quantize_mx (or fq_quantize_mx_static) with the same L = M*N:
+ *
+ *     C[t, o] = sum_i  A_hat[t, i] * W_hat[o, i],   X_hat[r, i] = e2m1(code) * 2^(byte - 127)
+ *
+ * with byte the E8M0 scale of group i / 32 of row r. It runs on the tensor cores' block-scaled
+ * FP4 MMA (kind::mxf4, one E8M0 scale per 32 elements), which reads the codes and scale bytes
+ * as the operator stores them. Products of E2M1 values and powers of two are exact; the sum
+ * is accumulated in float32 (order unspecified).
+ *   T, O       rows of A and of W, in [1, 262144]
+ *   L          elements per row, a multiple of 32 in [32, 65536]
+ *   a_fp4      [T, L/2] bytes, 16-byte aligned; a_scale_e8m0 [T, ceilDiv(L, 64), 2] bytes
+ *   w_fp4      [O, L/2] bytes, 16-byte aligned; w_scale_e8m0 [O, ceilDiv(L, 64), 2] bytes
+ *   C          [T, O] float32, row-major (4-byte aligned; O % 4 == 0 with a 16-byte aligned C
+ *              takes the vector stores)
+ *   status     a device word, or NULL: a bounded wait that gives up ORs a nonzero code into
+ *              it and leaves C undefined (with NULL nothing reports that)
+ * Allocates nothing; asynchronous on stream. Errors: FQ_ERR_NULLPTR (a_fp4, a_scale_e8m0,
+ * w_fp4, w_scale_e8m0, C), FQ_ERR_INVALID (a size out of range, L % 32 != 0, misaligned
+ * pointer), FQ_ERR_CUDA. */
+FQ_API fq_status fq_mx_matmul(int64_t T, int64_t O, int64_t L, const void *a_fp4,
+                              const uint8_t *a_scale_e8m0, const void *w_fp4,
+                              const uint8_t *w_scale_e8m0, float *C, uint32_t *status,
+                              struct CUstream_st *stream);
+
 /* Per-group mode (as fq_quantize_mx) for callers that cannot allocate device memory.
  * The paper has no counterpart: this entry point is an addition of this library.
  *

@@ -31,6 +31,7 @@ _SIGNATURES = {
     "fq_quantize_mx": (_int, [_vp, _vp, _vp, _vp, _dbl, _vp, _vp, _vp]),
     "fq_debug_rotate": (_int, [_vp, _vp, _vp, _vp, _vp, _vp]),
     "fq_quantize_mx_static": (_int, [_i64, _i64, _i64, _int, _vp, _vp, _vp, _dbl, _vp, _vp, _vp]),
+    "fq_mx_matmul": (_int, [_i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fq_static_device_status": (_int, [ctypes.POINTER(ctypes.c_uint32)]),
     "fq_static_debug_arm_stall": (_int, [_dbl]),
     "fq_set_kernel": (_int, [_vp, _int]),

@@ -190,6 +190,27 @@ fq_status fq_debug_rotate(fq_handle* h, const void* x, const void* P1, const voi
                 reinterpret_cast<cudaStream_t>(stream));
 }
 
+fq_status fq_mx_matmul(int64_t T, int64_t O, int64_t L, const void* a_fp4, const uint8_t* a_scale_e8m0,
+                       const void* w_fp4, const uint8_t* w_scale_e8m0, float* C, uint32_t* status,
+                       struct CUstream_st* stream) {
+  if (a_fp4 == nullptr || a_scale_e8m0 == nullptr || w_fp4 == nullptr || w_scale_e8m0 == nullptr ||
+      C == nullptr)
+    return FQ_ERR_NULLPTR;
+  // L is the flattened token M*N of the operator (M, N in [1, 256]), whole groups of 32;
+  // T and O are token counts (page: K in [1, 262144])
+  if (T < 1 || T > 262144 || O < 1 || O > 262144 || L < 32 || L > 65536 || L % 32 != 0)
+    return FQ_ERR_INVALID;
+  if (!aligned(a_fp4, 16) || !aligned(w_fp4, 16) || !aligned(C, 4) || (status && !aligned(status, 4)))
+    return FQ_ERR_INVALID;
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  fq::MxGemmParams p{a_fp4, a_scale_e8m0, w_fp4, w_scale_e8m0, C, status, T, O, L};
+  e = fq::launch_mxgemm(p, sms, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FQ_OK : cuda_fail(e);
+}
+
 fq_status fq_set_kernel(fq_handle* h, fq_kernel kernel) {
   if (h == nullptr) return FQ_ERR_NULLPTR;
   if (kernel != FQ_KERNEL_AUTO && kernel != FQ_KERNEL_GENERAL && kernel != FQ_KERNEL_TCGEN05)

@@ -57,6 +57,19 @@ bool tc_supported(int64_t K, int M, int N);
 // The one decoding used by every per-group entry point.
 bool mx_rule_from(double dst_type_max, MxRule* rule);
 
+// Block-scaled FP4 x FP4 contraction of two per-group outputs (see fq_mxgemm.cu):
+// C [T, O] float32 = A_hat [T, L] . W_hat [O, L]^T.
+struct MxGemmParams {
+  const void* a_codes;      // [T, L/2] bytes, 16-byte aligned
+  const uint8_t* a_scales;  // [T, 2*ceilDiv(L,64)] E8M0 bytes
+  const void* w_codes;      // [O, L/2]
+  const uint8_t* w_scales;  // [O, 2*ceilDiv(L,64)]
+  float* C;                 // [T, O]
+  uint32_t* status;         // bounded-wait status word, or nullptr
+  int64_t T, O, L;
+};
+cudaError_t launch_mxgemm(const MxGemmParams& p, int num_sms, cudaStream_t stream);
+
 // Keeps a CUDA error code for fq_last_cuda_error() (thread-local).
 void record_cuda_error(int e);
 cudaError_t launch_tc(const TcParams& p, bool fp16_in, int num_sms, cudaStream_t stream);
