@@ -19,8 +19,9 @@
 // row, one 128-byte swizzle atom). Roles, 384 threads:
 //   warp 0       TMA producer: code tiles of A (128 rows) and W (256 rows) into a 4-stage ring
 //   warp 1       MMA issuer (owns the TMEM allocation): four K = 64 MMAs per stage
-//   warps 4-7    scale warpgroup: per stage, reads the E8M0 words of the tile's rows from
-//                global memory and writes them into that stage's scale columns of TMEM
+//   warps 4-7    scale warpgroup: stages the E8M0 words of the tile's rows in shared memory
+//                with cp.async, four stages ahead, and writes each stage's words into that
+//                stage's scale columns of TMEM
 //   warps 8-11   epilogue: reads the float32 accumulator out of TMEM and stores C
 // Scale layout in TMEM (what the MMA reads): for a pair of K = 64 steps (four groups of
 // 32), row r of an operand with R rows has its four scale bytes in one 32-bit word at
@@ -58,7 +59,14 @@ constexpr int kSfaCols = 2 * (kBM / 32);  // two K pairs per stage, one column p
 constexpr int kSfbCols = 2 * (kBN / 32);
 constexpr int kSfCols = kSfaCols + kSfbCols;  // 24
 static_assert(kColSf + kStages * kSfCols <= kTmemCols, "TMEM columns");
-constexpr int kSmem = kStages * kStageBytes + 1024 /*barriers*/ + 1024 /*alignment*/;
+// Scale words staged in shared memory by the scale warpgroup with cp.async, kSfPrefetch
+// stages ahead of the one it writes to TMEM: one slot = 8 bytes (the stage's 8 groups) for
+// each of the tile's 128 + 256 rows.
+constexpr int kSfSlots = 6, kSfPrefetch = 4;
+constexpr int kSfSlotBytes = (kBM + kBN) * 8;
+constexpr int kOffSf = kStages * kStageBytes;
+constexpr int kSmem = kOffSf + kSfSlots * kSfSlotBytes + 1024 /*barriers*/ + 1024 /*alignment*/;
+static_assert(kSfPrefetch + 2 <= kSfSlots, "a slot is rewritten two stages after it was read");
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 
 enum : uint32_t {
@@ -85,6 +93,7 @@ struct GemmParams {
   int64_t T, O, L;
   int64_t sf_stride;   // scale bytes per row: 2 * ceilDiv(L, 64)
   int tiles_n, num_tiles, nk;
+  int sf_async;        // scale rows 8-byte aligned: staged with cp.async
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -234,7 +243,7 @@ mxgemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
               const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Bars* bars = reinterpret_cast<Bars*>(smem + kStages * kStageBytes);
+  Bars* bars = reinterpret_cast<Bars*>(smem + kOffSf + kSfSlots * kSfSlotBytes);
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -349,16 +358,69 @@ mxgemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
     // scale warps: warp q writes lanes 32q .. 32q + 31 (its sub-partition); lane i of every
     // sub-partition holds rows i, i + 32, ... of both operands (the MMA's layout)
     const int q = warp - kWarpSf0;
+    const int st = threadIdx.x - kWarpSf0 * 32;  // 0 .. 127 within the scale warpgroup
     const uint32_t t_lane = tmem + (uint32_t(q * 32) << 16);
-    int it = 0;
-    bool ok = true;
-    for (int i = 0; ok && i < n_local; ++i) {
+    const int n_it = n_local * p.nk;
+    // every scale warp runs every iteration (and every named barrier) to the end, also after
+    // a failed wait: a warp that left early would leave the others at the barrier
+    bool dead = false;
+    auto tile_rows = [&](int it, int64_t* m0, int64_t* n0, int* kb) {
+      const int i = it / p.nk;
+      *kb = it - i * p.nk;
       const int tile = int(blockIdx.x) + i * int(gridDim.x);
-      const int64_t m0 = int64_t(tile / p.tiles_n) * kBM, n0 = int64_t(tile % p.tiles_n) * kBN;
-      for (int kb = 0; kb < p.nk; ++kb, ++it) {
-        const int s = it % kStages;
-        // load before waiting: the global reads overlap the MMAs still using the slot
-        uint32_t va[kSfaCols], vb[kSfbCols];
+      *m0 = int64_t(tile / p.tiles_n) * kBM;
+      *n0 = int64_t(tile % p.tiles_n) * kBN;
+    };
+    // stage `it`'s 8-byte scale words of rows m0 + st (A) and n0 + st, n0 + 128 + st (W)
+    auto issue = [&](int it) {
+      if (p.sf_async && it < n_it) {
+        int64_t m0, n0;
+        int kb;
+        tile_rows(it, &m0, &n0, &kb);
+        const int64_t g0 = int64_t(kb) * 8;
+        const uint32_t valid = g0 < p.sf_stride ? 8u : 0u;  // the stride is a multiple of 8 here
+        const uint32_t slot = sbase + kOffSf + uint32_t((it % kSfSlots) * kSfSlotBytes);
+        const int64_t rows[3] = {m0 + st, n0 + st, n0 + 128 + st};
+        const uint8_t* bases[3] = {p.a_scales, p.w_scales, p.w_scales};
+        const int64_t lim[3] = {p.T, p.O, p.O};
+        const uint32_t dsts[3] = {slot + uint32_t(st * 8), slot + uint32_t((kBM + st) * 8),
+                                  slot + uint32_t((kBM + 128 + st) * 8)};
+#pragma unroll
+        for (int r = 0; r < 3; ++r) {
+          const bool in = rows[r] < lim[r];
+          const uint8_t* src = bases[r] + (in ? rows[r] * p.sf_stride + (valid ? g0 : 0) : 0);
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dsts[r]), "l"(src),
+                       "r"(in ? valid : 0u)
+                       : "memory");
+        }
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    for (int d = 0; d < kSfPrefetch; ++d) issue(d);
+    for (int it = 0; it < n_it; ++it) {
+      const int s = it % kStages;
+      issue(it + kSfPrefetch);
+      uint32_t va[kSfaCols], vb[kSfbCols];
+      if (p.sf_async) {
+        asm volatile("cp.async.wait_group %0;" ::"n"(kSfPrefetch) : "memory");
+        asm volatile("bar.sync 1, 128;" ::: "memory");  // every thread's copies of this stage landed
+        const uint8_t* slot = smem + kOffSf + (it % kSfSlots) * kSfSlotBytes;
+#pragma unroll
+        for (int j = 0; j < kBM / 32; ++j) {
+          const uint2 w = *reinterpret_cast<const uint2*>(slot + (j * 32 + lane) * 8);
+          va[j] = w.x;
+          va[kBM / 32 + j] = w.y;
+        }
+#pragma unroll
+        for (int j = 0; j < kBN / 32; ++j) {
+          const uint2 w = *reinterpret_cast<const uint2*>(slot + (kBM + j * 32 + lane) * 8);
+          vb[j] = w.x;
+          vb[kBN / 32 + j] = w.y;
+        }
+      } else {
+        int64_t m0, n0;
+        int kb;
+        tile_rows(it, &m0, &n0, &kb);
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const int64_t g0 = int64_t(kb) * 8 + 4 * c;
@@ -369,27 +431,27 @@ mxgemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
           for (int j = 0; j < kBN / 32; ++j)
             vb[c * (kBN / 32) + j] = load_sf_word(p.w_scales, p.O, n0 + j * 32 + lane, p.sf_stride, g0);
         }
-        if (it >= kStages && !warp_wait(&bars->empty[s], ((it / kStages) - 1) & 1, bars, p.status, kStEmpty)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t col = t_lane + kColSf + uint32_t(s * kSfCols);
-        tmem_st8(col, va);
-        tmem_st16(col + kSfaCols, vb);
-        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      }
+      if (dead) continue;
+      if (it >= kStages && !warp_wait(&bars->empty[s], ((it / kStages) - 1) & 1, bars, p.status, kStEmpty)) {
+        dead = true;
+        // publish every stage once, so the MMA warp is never left waiting on this warp
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->sf_full[s]);
+        if (lane == 0)
+          for (int s2 = 0; s2 < kStages; ++s2) mbar_arrive(&bars->sf_full[s2]);
+        continue;
       }
-    }
-    if (!ok) {
-      // publish every later stage once, so the MMA warp is never left waiting on this warp
+      tc_fence_after();
+      const uint32_t col = t_lane + kColSf + uint32_t(s * kSfCols);
+      tmem_st8(col, va);
+      tmem_st16(col + kSfaCols, vb);
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
       __syncwarp();
-      if (lane == 0)
-        for (int s = 0; s < kStages; ++s) mbar_arrive(&bars->sf_full[s]);
+      if (lane == 0) mbar_arrive(&bars->sf_full[s]);
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp >= kWarpEpi0 && warp < kWarpEpi0 + 4) {
     const int q = warp - kWarpEpi0;
     const uint32_t t_lane = tmem + (uint32_t(q * 32) << 16);
@@ -489,6 +551,8 @@ cudaError_t launch_mxgemm(const MxGemmParams& g, int num_sms, cudaStream_t strea
   p.tiles_n = int((g.O + kBN - 1) / kBN);
   p.num_tiles = int((g.T + kBM - 1) / kBM) * p.tiles_n;
   p.nk = int((g.L / 2 + kBKBytes - 1) / kBKBytes);
+  p.sf_async = (p.sf_stride % 8) == 0 && (reinterpret_cast<uintptr_t>(g.a_scales) & 7u) == 0 &&
+               (reinterpret_cast<uintptr_t>(g.w_scales) & 7u) == 0;
   cudaError_t e = cudaFuncSetAttribute(mxgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
