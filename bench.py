@@ -52,6 +52,8 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
+    p.add_argument("--no-consumer", action="store_true",
+                   help="skip the consumer FP4 x FP4 GEMM leg (timed apart from the step)")
     return p.parse_args(argv)
 
 
@@ -229,6 +231,62 @@ def bounded_oracle_sample(w, seed, target_s=12.0, min_tokens=16, max_tokens=4096
         dt = run(n)
     threads = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
     return n / dt, n, dt, threads
+
+
+FP4_PER_BF16 = 4.0  # nominal dense FP4 / bf16 tensor rate on B200 (9 / 2.25 PFLOP/s)
+
+
+def consumer_gemm_leg(w, dev, steps, bf16_tflops, peak_src, O=4096):
+    """Times fq_mx_matmul (the consumer contraction of two per-group outputs) on operands of
+    the workload's row length L = M*N: activations [T, L] with T = min(K, 8192), weights
+    [O, L], seeded random E2M1 codes and E8M0 bytes in [120, 133] drawn on the device. It is
+    timed apart from the step (it is not part of the fused operator). Returns a dict with
+    the time, TFLOP/s and the roofline against the FP4 dense peak, taken as the bf16 peak
+    times the nominal FP4 / bf16 ratio."""
+    import ctypes
+    from rotation_bit_quantization_token_b200 import _lib
+    lib = _lib.load()
+    L = w.M * w.N
+    T = min(w.K, 8192)
+    g = torch.Generator(device=dev).manual_seed(0)
+    S = 2 * (-(-L // 64))
+    a = torch.randint(0, 256, (T, L // 2), dtype=torch.uint8, device=dev, generator=g)
+    wt = torch.randint(0, 256, (O, L // 2), dtype=torch.uint8, device=dev, generator=g)
+    sa = torch.randint(120, 134, (T, S), dtype=torch.uint8, device=dev, generator=g)
+    sw = torch.randint(120, 134, (O, S), dtype=torch.uint8, device=dev, generator=g)
+    C = torch.empty((T, O), dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    vp = ctypes.c_void_p
+
+    def call():
+        st = lib.fq_mx_matmul(T, O, L, vp(a.data_ptr()), vp(sa.data_ptr()), vp(wt.data_ptr()),
+                              vp(sw.data_ptr()), vp(C.data_ptr()), vp(status.data_ptr()),
+                              vp(stream.cuda_stream))
+        if st != 0:
+            raise SystemExit(f"fq_mx_matmul failed: {st}")
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for e0, e1 in evs:
+        e0.record(stream)
+        call()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if int(status.item()) != 0:
+        raise SystemExit(f"fq_mx_matmul status {int(status.item())}")
+    ms = float(np.mean([e0.elapsed_time(e1) for e0, e1 in evs]))
+    tflops = 2.0 * T * O * L / (ms / 1e3) / 1e12
+    peak = bf16_tflops * FP4_PER_BF16
+    return {"op": "fq_mx_matmul", "shape": {"T": T, "O": O, "L": L}, "kernel_ms": ms,
+            "value": tflops, "unit": "TFLOP/s", "launches": steps,
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": tflops / peak,
+                         "peak_source": f"{peak_src} bf16 dense x {FP4_PER_BF16:g} (nominal FP4 / bf16 ratio)"},
+            "data": "seeded random E2M1 codes, E8M0 bytes 120-133"}
 
 
 # ----------------------------------------------------------------------------------------
@@ -431,6 +489,10 @@ def run_ours(args, rank, world, local):
                "h2d_bytes_per_step": pipe.h2d_bytes(), "d2h_bytes_per_step": pipe.d2h_bytes(),
                "ms_per_step": e_ms / e_steps}
 
+    consumer = None
+    if rank == 0 and world == 1 and not args.no_consumer:
+        consumer = consumer_gemm_leg(w, dev, max(3, min(args.steps, 10)), bf16_tflops, peak_src)
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -460,6 +522,7 @@ def run_ours(args, rank, world, local):
             "cpu_baseline": cpu,
             "e2e": e2e,
             "clocks": clock_info,
+            "consumer_gemm": consumer,
             "kernel_source": src_hash,
             "library": os.path.relpath(fqlib._lib.LIB_PATH, ROOT),
         }

@@ -98,7 +98,7 @@ bool fq::mx_rule_from(double d, fq::MxRule* r) {
   else if (d == 7.0) r->mode = fq::kMxMantissa7;
   else r->mode = fq::kMxRatio;
   r->dst_max = float(d);
-  r->inv_dst = d > 0.0 ? float(1.0 / d) : 0.0f;
+  r->inv_dst = d > 0.0 ? float(1.0 / double(float(d))) : 0.0f;
   return true;
 }
 

@@ -247,6 +247,48 @@ __device__ __forceinline__ void mma_ts_e(uint32_t d, uint32_t a_tmem, uint64_t b
       "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
+// Stage B of one 16-column block: the hi MMA (A at a_hi, accumulate flag acc_first) then
+// the lo MMA (A 8 columns further, always accumulating), both with B = b_desc, under one
+// election: the issuing warp shares its sub-partition with busy epilogue warps, so every
+// instruction it saves brings the next MMA to the tensor pipe sooner.
+__device__ __forceinline__ void mma_ts_block_e(uint32_t d, uint32_t a_hi, uint64_t b, uint32_t idesc,
+                                               uint32_t acc_first) {
+  asm volatile(
+      "{\n\t.reg .pred p, q, e;\n\t.reg .b32 r, a1;\n\t"
+      "elect.sync r|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 q, %4, %4;\n\t"
+      "add.u32 a1, %1, 8;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], %2, %3, q;\n\t}" ::"r"(d),
+      "r"(a_hi), "l"(b), "r"(idesc), "r"(acc_first)
+      : "memory");
+}
+// Stage A of one tile as eight K = 16 MMAs under one election: A = BD(P1) in TMEM at a
+// (8 columns per K step), B = the x tile at b_desc (2048 bytes per K step, 128 in the
+// descriptor's 16-byte units); the first MMA overwrites D.
+__device__ __forceinline__ void mma_ts_stage_a_e(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred f, t, e;\n\t.reg .b32 r, a1, a2, a3, a4, a5, a6, a7;\n\t"
+      ".reg .b64 b1, b2, b3, b4, b5, b6, b7;\n\t"
+      "elect.sync r|e, 0xffffffff;\n\t"
+      "setp.ne.b32 f, %1, %1;\n\t"
+      "setp.eq.b32 t, %1, %1;\n\t"
+      "add.u32 a1, %1, 8;\n\tadd.u32 a2, %1, 16;\n\tadd.u32 a3, %1, 24;\n\tadd.u32 a4, %1, 32;\n\t"
+      "add.u32 a5, %1, 40;\n\tadd.u32 a6, %1, 48;\n\tadd.u32 a7, %1, 56;\n\t"
+      "add.s64 b1, %2, 128;\n\tadd.s64 b2, %2, 256;\n\tadd.s64 b3, %2, 384;\n\tadd.s64 b4, %2, 512;\n\t"
+      "add.s64 b5, %2, 640;\n\tadd.s64 b6, %2, 768;\n\tadd.s64 b7, %2, 896;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, f;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b2, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b3, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a4], b4, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a5], b5, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a6], b6, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a7], b7, %3, t;\n\t}" ::"r"(d),
+      "r"(a), "l"(b), "r"(idesc)
+      : "memory");
+}
 __device__ __forceinline__ void mma_commit_e(uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
@@ -412,7 +454,9 @@ __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cas
 // ------------------------------------------------------------------------------------
 // the kernel
 // ------------------------------------------------------------------------------------
-template <int N, bool kF16, int kMode>
+// kRatio (per-group mode only): the group rule is case 3 (a separate instantiation, so that
+// the kernels of cases 1 and 2 carry none of its code)
+template <int N, bool kF16, int kMode, bool kRatio>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
   using G = Geo<N>;
@@ -590,12 +634,11 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
         tc_fence_after();
         const uint32_t d = tmem + uint32_t(sa * N);
         const uint64_t x_desc = desc64(sbase + G::kOffX + s * G::kXStage, 16384);
+        if constexpr (G::kP1Tmem) {
+          mma_ts_stage_a_e(d, tmem + G::kP1Col, x_desc, kIdA);
+        } else {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          if constexpr (G::kP1Tmem)
-            mma_ts_e(d, tmem + G::kP1Col + uint32_t(kk * 8), x_desc + uint64_t((kk * 2048) >> 4), kIdA,
-                     kk > 0 ? 1u : 0u);
-          else
+          for (int kk = 0; kk < 8; ++kk)
             mma_ss_e(d, p1_desc + uint64_t(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
                      x_desc + uint64_t((kk * 2048) >> 4), kIdA, kk > 0 ? 1u : 0u);
         }
@@ -619,13 +662,10 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 2 * g; kk < 2 * g + 2 && kk < G::kBlocks; ++kk) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-              mma_ts_e(d, a0 + uint32_t(kk * 16 + h * 8),
-                       p2_desc + uint64_t(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4), kIdB,
-                       (h | kk) != 0 ? 1u : 0u);
-          }
+          for (int kk = 2 * g; kk < 2 * g + 2 && kk < G::kBlocks; ++kk)
+            mma_ts_block_e(d, a0 + uint32_t(kk * 16),
+                           p2_desc + uint64_t(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4), kIdB,
+                           kk != 0 ? 1u : 0u);
         }
         if (!ok) break;
         mma_commit_e(&bars->db_full[b % kEpi]);
@@ -866,35 +906,64 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
           for (int sg = 0; sg < NS; ++sg) Fseg[sg] = inv * fcrow;
         } else {
           named_bar(bar_id, 128);
+          // bytes by each rule's common path; a ratio-rule group next to a power of two is
+          // decided again exactly, by the whole warp when any lane has one (rare)
+          constexpr int GR = (N % 32) == 0 ? NS / 2 : (N - 16) / 32 + 1;  // groups met by a row
+          float gam[GR];
+          uint32_t gb[GR];
+          const bool odd = (row & 1) != 0;
+          if constexpr ((N % 32) == 0) {
+#pragma unroll
+            for (int gi = 0; gi < GR; ++gi) gam[gi] = fmaxf(smax[2 * gi], smax[2 * gi + 1]) * fcrow;
+          } else {
+            // groups of 32 straddle rows: the last 16 columns of an even row and the first
+            // 16 of the next row form one group (the pair sits in adjacent lanes); it is
+            // group GR - 1 here
+            constexpr int GF = GR - 1;  // full groups per row
+            const float part = (odd ? smax[0] : smax[NS - 1]) * fcrow;
+            const float other = __shfl_xor_sync(0xffffffffu, part, 1);
+#pragma unroll
+            for (int gi = 0; gi < GF; ++gi)
+              gam[gi] = (odd ? fmaxf(smax[2 * gi + 1], smax[2 * gi + 2]) : fmaxf(smax[2 * gi], smax[2 * gi + 1])) * fcrow;
+            gam[GF] = fmaxf(part, other);
+          }
+          bool any_rare = false;
+#pragma unroll
+          for (int gi = 0; gi < GR; ++gi) {
+            bool r;
+            gb[gi] = mx_byte_common<kRatio ? kMxRatio : 0>(gam[gi], p.rule, &r);
+            any_rare |= r;
+          }
+          if constexpr (kRatio) {
+            if (__any_sync(0xffffffffu, any_rare)) {
+#pragma unroll
+              for (int gi = 0; gi < GR; ++gi) {
+                bool r;
+                mx_byte_common<kMxRatio>(gam[gi], p.rule, &r);
+                if (r) gb[gi] = mx_byte_rare(gam[gi], p.rule);
+              }
+            }
+          }
           uint8_t* s_scale = s_out + G::kCodeBytes;
           if constexpr ((N % 32) == 0) {
 #pragma unroll
-            for (int gi = 0; gi < NS / 2; ++gi) {
-              const MxScale ms = mx_scale<true>(fmaxf(smax[2 * gi], smax[2 * gi + 1]) * fcrow, p.rule);
-              const float F = exp2i(127 - int(ms.byte) + crow);
+            for (int gi = 0; gi < GR; ++gi) {
+              const float F = exp2i(127 - int(gb[gi]) + crow);
               Fseg[2 * gi] = F;
               Fseg[2 * gi + 1] = F;
-              s_scale[row * (N / 32) + gi] = uint8_t(ms.byte);
+              s_scale[row * (N / 32) + gi] = uint8_t(gb[gi]);
             }
           } else {
-            // groups of 32 straddle rows: the last 16 columns of an even row and the first
-            // 16 of the next row form one group (the pair sits in adjacent lanes)
-            constexpr int GF = (N - 16) / 32;  // full groups per row
-            const bool odd = (row & 1) != 0;
-            const float part = (odd ? smax[0] : smax[NS - 1]) * fcrow;
-            const float other = __shfl_xor_sync(0xffffffffu, part, 1);
-            const MxScale mst = mx_scale<true>(fmaxf(part, other), p.rule);
-            const float Fst = exp2i(127 - int(mst.byte) + crow);
+            constexpr int GF = GR - 1;
+            const float Fst = exp2i(127 - int(gb[GF]) + crow);
             const int pair_base = (row >> 1) * (N / 16);
             float Ff[GF];
 #pragma unroll
             for (int gi = 0; gi < GF; ++gi) {
-              const float a = odd ? fmaxf(smax[2 * gi + 1], smax[2 * gi + 2]) : fmaxf(smax[2 * gi], smax[2 * gi + 1]);
-              const MxScale ms = mx_scale<true>(a * fcrow, p.rule);
-              Ff[gi] = exp2i(127 - int(ms.byte) + crow);
-              s_scale[pair_base + (odd ? GF + 1 : 0) + gi] = uint8_t(ms.byte);
+              Ff[gi] = exp2i(127 - int(gb[gi]) + crow);
+              s_scale[pair_base + (odd ? GF + 1 : 0) + gi] = uint8_t(gb[gi]);
             }
-            if (!odd) s_scale[pair_base + GF] = uint8_t(mst.byte);
+            if (!odd) s_scale[pair_base + GF] = uint8_t(gb[GF]);
 #pragma unroll
             for (int sg = 0; sg < NS; ++sg) {
               const float fe = (sg == NS - 1) ? Fst : Ff[sg >> 1];
@@ -950,7 +1019,7 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-template <int N, bool kF16, int kMode>
+template <int N, bool kF16, int kMode, bool kRatio = false>
 cudaError_t launch_n(const TcParams& p, int num_sms, cudaStream_t stream) {
   using G = Geo<N>;
   auto enc = get_encode();
@@ -965,7 +1034,7 @@ cudaError_t launch_n(const TcParams& p, int num_sms, cudaStream_t stream) {
                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  auto kern = tc_kernel<N, kF16, kMode>;
+  auto kern = tc_kernel<N, kF16, kMode, kRatio>;
   // The register split is sized for kLaunchRegs per thread; a kernel built with fewer
   // would make setmaxnreg.inc wait for registers that do not exist, so refuse it.
   cudaFuncAttributes fa;
@@ -985,7 +1054,11 @@ cudaError_t launch_mode(const TcParams& p, bool f16, int sms, cudaStream_t s) {
   if (p.mode == kModePerToken)
     return f16 ? launch_n<N, true, kModePerToken>(p, sms, s) : launch_n<N, false, kModePerToken>(p, sms, s);
   if (p.mode == kModeMx)
-    return f16 ? launch_n<N, true, kModeMx>(p, sms, s) : launch_n<N, false, kModeMx>(p, sms, s);
+  {
+    if (p.rule.mode == kMxRatio)
+      return f16 ? launch_n<N, true, kModeMx, true>(p, sms, s) : launch_n<N, false, kModeMx, true>(p, sms, s);
+    return f16 ? launch_n<N, true, kModeMx, false>(p, sms, s) : launch_n<N, false, kModeMx, false>(p, sms, s);
+  }
   return f16 ? launch_n<N, true, kModeRotate>(p, sms, s) : launch_n<N, false, kModeRotate>(p, sms, s);
 }
 
