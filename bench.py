@@ -54,6 +54,8 @@ def parse_args(argv=None):
     p.add_argument("--no-clocks", action="store_true")
     p.add_argument("--no-consumer", action="store_true",
                    help="skip the consumer FP4 x FP4 GEMM leg (timed apart from the step)")
+    p.add_argument("--consumer-only", action="store_true",
+                   help="time only the consumer GEMM leg and print its object (for profiling)")
     return p.parse_args(argv)
 
 
@@ -371,6 +373,12 @@ def run_ours(args, rank, world, local):
     w = WORKLOADS[args.workload]
     if args.tokens:
         w = w.with_tokens(args.tokens)
+    if args.consumer_only:
+        hbm_gbs, bf16_tflops, peak_src = load_peaks()
+        if rank == 0:
+            print(json.dumps(consumer_gemm_leg(w, dev, max(1, args.steps), bf16_tflops, peak_src)),
+                  flush=True)
+        return 0
     # cpu baseline first (rank 0 at N = 1 only), while nothing runs on the GPU
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
