@@ -500,6 +500,19 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
+  // the producer issues its first round of x loads now: nothing below writes the x ring, so
+  // their latency overlaps the rest of the prologue (a small launch spends a good part of its
+  // time there)
+  const int n_early = (warp == kWarpProducer && lane == 0 && !p.stall_loads && int(blockIdx.x) < num_tiles)
+                          ? min((num_tiles - 1 - int(blockIdx.x)) / int(gridDim.x) + 1, G::kStages)
+                          : 0;
+  for (int i = 0; i < n_early; ++i) {
+    mbar_arrive_expect_tx(&bars->x_full[i], G::kXStage);
+#pragma unroll
+    for (int a = 0; a < G::kAtoms; ++a)
+      tma_load_2d(sbase + G::kOffX + i * G::kXStage + a * 16384, &tmap, a * 64,
+                  (int(blockIdx.x) + i * int(gridDim.x)) * 128, &bars->x_full[i]);
+  }
   float p2max = 0.0f;
 #pragma unroll
   for (int w = 0; w < kThreads / 32; ++w) p2max = fmaxf(p2max, bars->wmax[w]);
@@ -582,11 +595,11 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     // (test hook) with stall_loads the producer issues nothing, so the first stage-A wait can
     // only end by running out
     if (lane == 0 && !p.stall_loads) {
-      int i = 0;
       int last_i[G::kStages];
 #pragma unroll
-      for (int s = 0; s < G::kStages; ++s) last_i[s] = -1;
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
+      for (int s = 0; s < G::kStages; ++s) last_i[s] = s < n_early ? s : -1;
+      int i = n_early;  // the first round went out in the prologue
+      for (int tile = blockIdx.x + n_early * gridDim.x; tile < num_tiles; tile += gridDim.x, ++i) {
         const int s = i % G::kStages;
         if (!wait_bounded(&bars->x_empty[s], ((i / G::kStages) & 1) ^ 1, bars, p.status, kStProducerEmpty)) break;
         mbar_arrive_expect_tx(&bars->x_full[s], G::kXStage);
