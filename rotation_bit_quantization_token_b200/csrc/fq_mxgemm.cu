@@ -18,17 +18,24 @@
 // TMEM lanes, W rows along the MMA's N), K in stages of 256 elements (128 code bytes per
 // row, one 128-byte swizzle atom). Roles, 384 threads:
 //   warp 0       TMA producer: code tiles of A (128 rows) and W (256 rows) into a 4-stage ring
-//   warp 1       MMA issuer (owns the TMEM allocation): four K = 64 MMAs per stage
-//   warps 4-7    scale warpgroup: stages the E8M0 words of the tile's rows in shared memory
-//                with cp.async, four stages ahead, and writes each stage's words into that
-//                stage's scale columns of TMEM
+//   warp 1       MMA issuer (owns the TMEM allocation): per stage, six tcgen05.cp of the
+//                stage's scale words from shared memory into its scale columns of TMEM,
+//                then four K = 64 MMAs (the copies and MMAs of one thread run in issue order)
+//   warps 4-7    scale producer: reads the tile rows' E8M0 words (16 bytes of a row, two
+//                stages, per load, two loads ahead) and stores each stage's words into a
+//                scale slot in shared memory (an 8-slot ring of its own) in the order
+//                tcgen05.cp reads them
 //   warps 8-11   epilogue: reads the float32 accumulator out of TMEM and stores C
 // Scale layout in TMEM (what the MMA reads): for a pair of K = 64 steps (four groups of
 // 32), row r of an operand with R rows has its four scale bytes in one 32-bit word at
 // lane r % 32 of every 32-lane sub-partition, column (pair base) + r / 32; the first MMA of
 // the pair reads bytes 0-1, the second bytes 2-3 (selected by the scale-factor id). The
-// operator's scale bytes of groups 4c .. 4c + 3 of a row are one aligned 32-bit word, so
-// the words move unchanged.
+// operator's scale bytes of groups 4c .. 4c + 3 of a row are one 32-bit word, so the words
+// move unchanged; only their places change. A tcgen05.cp of shape 32x128b with .warpx4
+// writes 32 shared-memory rows of 16 bytes to lanes 0-31 of all four sub-partitions, four
+// columns wide, so one 512-byte block whose row l holds, at bytes 4j .. 4j + 3, the word of
+// operand row 32j + l fills four columns of that layout: two blocks per stage for A (one
+// per K pair), four for W (two per K pair).
 // Every wait is bounded in time; on expiry the kernel sets a bit in the caller's status
 // word (if one is given), lets every role leave, waits for its copies and MMAs, frees
 // TMEM and returns.
@@ -59,14 +66,18 @@ constexpr int kSfaCols = 2 * (kBM / 32);  // two K pairs per stage, one column p
 constexpr int kSfbCols = 2 * (kBN / 32);
 constexpr int kSfCols = kSfaCols + kSfbCols;  // 24
 static_assert(kColSf + kStages * kSfCols <= kTmemCols, "TMEM columns");
-// Scale words staged in shared memory by the scale warpgroup with cp.async, kSfPrefetch
-// stages ahead of the one it writes to TMEM: one slot = 8 bytes (the stage's 8 groups) for
-// each of the tile's 128 + 256 rows.
-constexpr int kSfSlots = 6, kSfPrefetch = 4;
-constexpr int kSfSlotBytes = (kBM + kBN) * 8;
+// Scale slot of a stage in shared memory: 512-byte blocks of 32 rows x 16 bytes, in the
+// order tcgen05.cp reads them: A groups 0-3, A groups 4-7, W rows 0-127 groups 0-3, W rows
+// 128-255 groups 0-3, W rows 0-127 groups 4-7, W rows 128-255 groups 4-7.
+constexpr int kSfBlockBytes = 512;
+constexpr int kSfSlotBytes = 6 * kSfBlockBytes;
+static_assert(kSfSlotBytes == (kBM + kBN) * 8, "8 scale bytes per row and stage");
+// The scale slots form their own ring, deeper than the code stages, so that the copies
+// (many small reads) have several stages of MMA time to land.
+constexpr int kSfStages = 8;
 constexpr int kOffSf = kStages * kStageBytes;
-constexpr int kSmem = kOffSf + kSfSlots * kSfSlotBytes + 1024 /*barriers*/ + 1024 /*alignment*/;
-static_assert(kSfPrefetch + 2 <= kSfSlots, "a slot is rewritten two stages after it was read");
+constexpr int kSmem = kOffSf + kSfStages * kSfSlotBytes + 1024 /*barriers*/ + 1024 /*alignment*/;
+static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 
 enum : uint32_t {
@@ -77,7 +88,8 @@ enum : uint32_t {
 struct Bars {
   uint64_t full[kStages];     // TMA bytes of stage s landed
   uint64_t empty[kStages];    // the MMAs that read stage s (codes and scale columns) completed
-  uint64_t sf_full[kStages];  // scale columns of stage s written (one arrive per scale warp)
+  uint64_t sf_full[kSfStages];   // scale slot j filled (one arrive per scale thread)
+  uint64_t sf_empty[kSfStages];  // the copies out of scale slot j completed
   uint64_t d_full;            // accumulator of the tile complete
   uint64_t d_empty;           // accumulator read out (one arrive per epilogue warp)
   uint64_t mma_done;
@@ -93,7 +105,7 @@ struct GemmParams {
   int64_t T, O, L;
   int64_t sf_stride;   // scale bytes per row: 2 * ceilDiv(L, 64)
   int tiles_n, num_tiles, nk;
-  int sf_async;        // scale rows 8-byte aligned: staged with cp.async
+  int sf_vec;          // scale rows 16-byte aligned: read 16 bytes (two stages) at a time
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -168,6 +180,15 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   return (uint64_t(hi) << 32) | lo;
 }
 
+// Shared-memory descriptor without swizzle: 8-row groups of 16-byte rows, 128 bytes apart
+// (rows contiguous), the source form of tcgen05.cp. The rows are one core matrix wide, so
+// only the 8-row-group stride is used; both offset fields carry it.
+__device__ __forceinline__ uint64_t plain_desc(uint32_t saddr) {
+  const uint32_t lo = (saddr >> 4) | ((128u >> 4) << 16);
+  const uint32_t hi = (128u >> 4) | (1u << 14);
+  return (uint64_t(hi) << 32) | lo;
+}
+
 // Instruction descriptor of kind::mxf4 with E8M0 scales, M = 128, N = kBN, both operands
 // K-major E2M1; the scale-factor ids (byte offset of the K pair's half) are set per MMA.
 __host__ __device__ constexpr uint32_t idesc_mxf4(uint32_t sf_id) {
@@ -179,38 +200,35 @@ __host__ __device__ constexpr uint32_t idesc_mxf4(uint32_t sf_id) {
          (sf_id << 29);            // A scale-factor id
 }
 
+// The three below are issued by one thread (the MMA warp's leader), so that the copies, the
+// MMAs and the commit that tracks them all belong to the same thread.
 __device__ __forceinline__ void mma_mxf4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
                                          uint32_t sfb, uint32_t acc) {
   asm volatile(
-      "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\t"
-      "elect.sync r|e, 0xffffffff;\n\t"
+      "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
       ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
       : "memory");
 }
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+// 32 rows x 16 bytes of shared memory to lanes 0-31 of every sub-partition, four columns.
+__device__ __forceinline__ void sf_copy(uint32_t taddr, uint64_t src) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src) : "memory");
+}
+__device__ __forceinline__ void mma_commit_one(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ bool elect_one() {
+  uint32_t e;
   asm volatile(
       "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
       "elect.sync r|e, 0xffffffff;\n\t"
-      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
-          smem_u32(bar))
-      : "memory");
+      "selp.u32 %0, 1, 0, e;\n\t}"
+      : "=r"(e));
+  return e != 0;
 }
 
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
-      "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
@@ -243,7 +261,7 @@ mxgemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
               const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Bars* bars = reinterpret_cast<Bars*>(smem + kOffSf + kSfSlots * kSfSlotBytes);
+  Bars* bars = reinterpret_cast<Bars*>(smem + kOffSf + kSfStages * kSfSlotBytes);
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -251,7 +269,10 @@ mxgemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->empty[s], 1);
-      mbar_init(&bars->sf_full[s], 4);
+    }
+    for (int j = 0; j < kSfStages; ++j) {
+      mbar_init(&bars->sf_full[j], 128);
+      mbar_init(&bars->sf_empty[j], 1);
     }
     mbar_init(&bars->d_full, 1);
     mbar_init(&bars->d_empty, 4);
@@ -308,6 +329,7 @@ mxgemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
     }
     __syncwarp();
   } else if (warp == kWarpMma) {
+    const bool leader = elect_one();
     int it = 0;
     bool ok = true;
     for (int i = 0; ok && i < n_local; ++i) {
@@ -315,34 +337,49 @@ mxgemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
       tc_fence_after();
       for (int kb = 0; kb < p.nk; ++kb, ++it) {
         const int s = it % kStages;
-        const uint32_t par = (it / kStages) & 1;
-        if (!warp_wait(&bars->full[s], par, bars, p.status, kStFull) ||
-            !warp_wait(&bars->sf_full[s], par, bars, p.status, kStSfFull)) {
+        const int j = it % kSfStages;
+        if (!warp_wait(&bars->full[s], (it / kStages) & 1, bars, p.status, kStFull) ||
+            !warp_wait(&bars->sf_full[j], (it / kSfStages) & 1, bars, p.status, kStSfFull)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t a_addr = sbase + s * kStageBytes;
-        const uint64_t a_desc = sw128_desc(a_addr);
-        const uint64_t b_desc = sw128_desc(a_addr + kABytes);
-        const uint32_t sfa_col = tmem + kColSf + uint32_t(s * kSfCols);
-        const uint32_t sfb_col = sfa_col + kSfaCols;
+        if (leader) {
+          const uint32_t a_addr = sbase + s * kStageBytes;
+          const uint64_t a_desc = sw128_desc(a_addr);
+          const uint64_t b_desc = sw128_desc(a_addr + kABytes);
+          const uint32_t sfa_col = tmem + kColSf + uint32_t(s * kSfCols);
+          const uint32_t sfb_col = sfa_col + kSfaCols;
+          const uint32_t slot = sbase + kOffSf + uint32_t(j * kSfSlotBytes);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t id = uint32_t(2 * (k & 1));  // byte offset of this K step in its pair's words
-          const uint32_t sfa = (sfa_col + uint32_t((k >> 1) * (kBM / 32))) | (id << 30);
-          const uint32_t sfb = (sfb_col + uint32_t((k >> 1) * (kBN / 32))) | (id << 30);
-          // 64 elements = 32 bytes further along K inside the swizzle atom
-          mma_mxf4(tmem + kColD, a_desc + uint64_t((k * 32) >> 4), b_desc + uint64_t((k * 32) >> 4),
-                   idesc_mxf4(id), sfa, sfb, (kb | k) != 0 ? 1u : 0u);
+          for (int pr = 0; pr < 2; ++pr) {  // K pair pr: groups 4pr .. 4pr + 3
+            sf_copy(sfa_col + uint32_t(pr * (kBM / 32)), plain_desc(slot + uint32_t(pr * kSfBlockBytes)));
+#pragma unroll
+            for (int hb = 0; hb < 2; ++hb)
+              sf_copy(sfb_col + uint32_t(pr * (kBN / 32) + 4 * hb),
+                      plain_desc(slot + uint32_t((2 + 2 * pr + hb) * kSfBlockBytes)));
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t id = uint32_t(2 * (k & 1));  // byte offset of this K step in its pair's words
+            const uint32_t sfa = (sfa_col + uint32_t((k >> 1) * (kBM / 32))) | (id << 30);
+            const uint32_t sfb = (sfb_col + uint32_t((k >> 1) * (kBN / 32))) | (id << 30);
+            // 64 elements = 32 bytes further along K inside the swizzle atom
+            mma_mxf4(tmem + kColD, a_desc + uint64_t((k * 32) >> 4), b_desc + uint64_t((k * 32) >> 4),
+                     idesc_mxf4(id), sfa, sfb, (kb | k) != 0 ? 1u : 0u);
+          }
+          mma_commit_one(&bars->empty[s]);
+          mma_commit_one(&bars->sf_empty[j]);
         }
-        mma_commit(&bars->empty[s]);
+        __syncwarp();
       }
       if (!ok) break;
-      mma_commit(&bars->d_full);
+      if (leader) mma_commit_one(&bars->d_full);
+      __syncwarp();
     }
     // every MMA issued here has completed before TMEM is released
-    mma_commit(&bars->mma_done);
+    if (leader) mma_commit_one(&bars->mma_done);
+    __syncwarp();
     if (lane == 0) {
       const uint32_t bd = smem_u32(&bars->mma_done);
       const uint64_t t0 = globaltimer();
@@ -355,103 +392,87 @@ mxgemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
     }
     __syncwarp();
   } else if (warp >= kWarpSf0 && warp < kWarpSf0 + 4) {
-    // scale warps: warp q writes lanes 32q .. 32q + 31 (its sub-partition); lane i of every
-    // sub-partition holds rows i, i + 32, ... of both operands (the MMA's layout)
-    const int q = warp - kWarpSf0;
-    const int st = threadIdx.x - kWarpSf0 * 32;  // 0 .. 127 within the scale warpgroup
-    const uint32_t t_lane = tmem + (uint32_t(q * 32) << 16);
-    const int n_it = n_local * p.nk;
-    // every scale warp runs every iteration (and every named barrier) to the end, also after
-    // a failed wait: a warp that left early would leave the others at the barrier
-    bool dead = false;
-    auto tile_rows = [&](int it, int64_t* m0, int64_t* n0, int* kb) {
-      const int i = it / p.nk;
-      *kb = it - i * p.nk;
+    // thread st carries row st of the A tile and rows st, 128 + st of the W tile: row 32c + l
+    // of an operand goes to row l, bytes 4c .. 4c + 3, of its block
+    const int st = threadIdx.x - kWarpSf0 * 32;
+    const uint32_t off = uint32_t(16 * (st & 31) + 4 * (st >> 5));
+    const uint8_t* bases[3] = {p.a_scales, p.w_scales, p.w_scales};
+    const int64_t lim[3] = {p.T, p.O, p.O};
+    auto tile_row = [&](int i, int r) {
       const int tile = int(blockIdx.x) + i * int(gridDim.x);
-      *m0 = int64_t(tile / p.tiles_n) * kBM;
-      *n0 = int64_t(tile % p.tiles_n) * kBN;
+      return r == 0 ? int64_t(tile / p.tiles_n) * kBM + st : int64_t(tile % p.tiles_n) * kBN + 128 * (r - 1) + st;
     };
-    // stage `it`'s 8-byte scale words of rows m0 + st (A) and n0 + st, n0 + 128 + st (W)
-    auto issue = [&](int it) {
-      if (p.sf_async && it < n_it) {
-        int64_t m0, n0;
-        int kb;
-        tile_rows(it, &m0, &n0, &kb);
-        const int64_t g0 = int64_t(kb) * 8;
-        const uint32_t valid = g0 < p.sf_stride ? 8u : 0u;  // the stride is a multiple of 8 here
-        const uint32_t slot = sbase + kOffSf + uint32_t((it % kSfSlots) * kSfSlotBytes);
-        const int64_t rows[3] = {m0 + st, n0 + st, n0 + 128 + st};
-        const uint8_t* bases[3] = {p.a_scales, p.w_scales, p.w_scales};
-        const int64_t lim[3] = {p.T, p.O, p.O};
-        const uint32_t dsts[3] = {slot + uint32_t(st * 8), slot + uint32_t((kBM + st) * 8),
-                                  slot + uint32_t((kBM + 128 + st) * 8)};
+    bool ok = true;
+    // one stage's words (groups 0-3 and 4-7 of the stage for the three rows) into scale slot
+    // j; the writer fences its stores for the async proxy, then arrives
+    auto put = [&](int it, const uint32_t (&w)[3][2]) {
+      const int j = it % kSfStages;
+      if (it >= kSfStages &&
+          !warp_wait(&bars->sf_empty[j], ((it / kSfStages) - 1) & 1, bars, p.status, kStEmpty)) {
+        ok = false;
+        return;
+      }
+      const uint32_t slot = sbase + kOffSf + uint32_t(j * kSfSlotBytes);
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
 #pragma unroll
         for (int r = 0; r < 3; ++r) {
-          const bool in = rows[r] < lim[r];
-          const uint8_t* src = bases[r] + (in ? rows[r] * p.sf_stride + (valid ? g0 : 0) : 0);
-          asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dsts[r]), "l"(src),
-                       "r"(in ? valid : 0u)
+          const int blk = r == 0 ? h : 2 + 2 * h + (r - 1);
+          asm volatile("st.shared.u32 [%0], %1;" ::"r"(slot + uint32_t(blk * kSfBlockBytes) + off), "r"(w[r][h])
                        : "memory");
         }
-      }
-      asm volatile("cp.async.commit_group;" ::: "memory");
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&bars->sf_full[j]);
     };
-    for (int d = 0; d < kSfPrefetch; ++d) issue(d);
-    for (int it = 0; it < n_it; ++it) {
-      const int s = it % kStages;
-      issue(it + kSfPrefetch);
-      uint32_t va[kSfaCols], vb[kSfbCols];
-      if (p.sf_async) {
-        asm volatile("cp.async.wait_group %0;" ::"n"(kSfPrefetch) : "memory");
-        asm volatile("bar.sync 1, 128;" ::: "memory");  // every thread's copies of this stage landed
-        const uint8_t* slot = smem + kOffSf + (it % kSfSlots) * kSfSlotBytes;
+    if (p.sf_vec) {
+      // 16 bytes of a row (the groups of two stages) per load, issued two units ahead of use;
+      // unit n = stages 2v, 2v + 1 of local tile n / upt (v = n % upt)
+      const int upt = (p.nk + 1) / 2;
+      const int n_units = n_local * upt;
+      auto load = [&](int n, uint4 (&b)[3]) {
+        if (n >= n_units) return;
+        const int i = n / upt;
+        const int64_t g0 = int64_t(n - i * upt) * 16;
 #pragma unroll
-        for (int j = 0; j < kBM / 32; ++j) {
-          const uint2 w = *reinterpret_cast<const uint2*>(slot + (j * 32 + lane) * 8);
-          va[j] = w.x;
-          va[kBM / 32 + j] = w.y;
+        for (int r = 0; r < 3; ++r) {
+          const int64_t row = tile_row(i, r);
+          b[r] = row < lim[r] ? __ldg(reinterpret_cast<const uint4*>(bases[r] + row * p.sf_stride + g0))
+                              : make_uint4(0u, 0u, 0u, 0u);
         }
-#pragma unroll
-        for (int j = 0; j < kBN / 32; ++j) {
-          const uint2 w = *reinterpret_cast<const uint2*>(slot + (kBM + j * 32 + lane) * 8);
-          vb[j] = w.x;
-          vb[kBN / 32 + j] = w.y;
+      };
+      auto store = [&](int n, const uint4 (&b)[3]) {
+        const int i = n / upt, v = n - i * upt;
+        const uint32_t w0[3][2] = {{b[0].x, b[0].y}, {b[1].x, b[1].y}, {b[2].x, b[2].y}};
+        put(i * p.nk + 2 * v, w0);
+        if (ok && 2 * v + 1 < p.nk) {
+          const uint32_t w1[3][2] = {{b[0].z, b[0].w}, {b[1].z, b[1].w}, {b[2].z, b[2].w}};
+          put(i * p.nk + 2 * v + 1, w1);
         }
-      } else {
-        int64_t m0, n0;
-        int kb;
-        tile_rows(it, &m0, &n0, &kb);
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int64_t g0 = int64_t(kb) * 8 + 4 * c;
-#pragma unroll
-          for (int j = 0; j < kBM / 32; ++j)
-            va[c * (kBM / 32) + j] = load_sf_word(p.a_scales, p.T, m0 + j * 32 + lane, p.sf_stride, g0);
-#pragma unroll
-          for (int j = 0; j < kBN / 32; ++j)
-            vb[c * (kBN / 32) + j] = load_sf_word(p.w_scales, p.O, n0 + j * 32 + lane, p.sf_stride, g0);
-        }
+      };
+      uint4 b0[3], b1[3];
+      load(0, b0);
+      load(1, b1);
+      for (int n = 0; ok && n < n_units; n += 2) {
+        store(n, b0);
+        load(n + 2, b0);
+        if (!ok || n + 1 >= n_units) break;
+        store(n + 1, b1);
+        load(n + 3, b1);
       }
-      if (dead) continue;
-      if (it >= kStages && !warp_wait(&bars->empty[s], ((it / kStages) - 1) & 1, bars, p.status, kStEmpty)) {
-        dead = true;
-        // publish every stage once, so the MMA warp is never left waiting on this warp
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0)
-          for (int s2 = 0; s2 < kStages; ++s2) mbar_arrive(&bars->sf_full[s2]);
-        continue;
-      }
-      tc_fence_after();
-      const uint32_t col = t_lane + kColSf + uint32_t(s * kSfCols);
-      tmem_st8(col, va);
-      tmem_st16(col + kSfaCols, vb);
-      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->sf_full[s]);
+    } else {
+      // any row stride or alignment: word by word, bytes past the row read as 0
+      int it = 0;
+      for (int i = 0; ok && i < n_local; ++i)
+        for (int kb = 0; ok && kb < p.nk; ++kb, ++it) {
+          uint32_t w[3][2];
+#pragma unroll
+          for (int r = 0; r < 3; ++r)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              w[r][h] = load_sf_word(bases[r], lim[r], tile_row(i, r), p.sf_stride, int64_t(kb) * 8 + 4 * h);
+          put(it, w);
+        }
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp >= kWarpEpi0 && warp < kWarpEpi0 + 4) {
     const int q = warp - kWarpEpi0;
     const uint32_t t_lane = tmem + (uint32_t(q * 32) << 16);
@@ -551,8 +572,8 @@ cudaError_t launch_mxgemm(const MxGemmParams& g, int num_sms, cudaStream_t strea
   p.tiles_n = int((g.O + kBN - 1) / kBN);
   p.num_tiles = int((g.T + kBM - 1) / kBM) * p.tiles_n;
   p.nk = int((g.L / 2 + kBKBytes - 1) / kBKBytes);
-  p.sf_async = (p.sf_stride % 8) == 0 && (reinterpret_cast<uintptr_t>(g.a_scales) & 7u) == 0 &&
-               (reinterpret_cast<uintptr_t>(g.w_scales) & 7u) == 0;
+  p.sf_vec = (p.sf_stride % 16) == 0 && (reinterpret_cast<uintptr_t>(g.a_scales) & 15u) == 0 &&
+             (reinterpret_cast<uintptr_t>(g.w_scales) & 15u) == 0;
   cudaError_t e = cudaFuncSetAttribute(mxgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
