@@ -75,6 +75,7 @@ static_assert(kSfSlotBytes == (kBM + kBN) * 8, "8 scale bytes per row and stage"
 // The scale slots form their own ring, deeper than the code stages, so that the copies
 // (many small reads) have several stages of MMA time to land.
 constexpr int kSfStages = 8;
+constexpr int kSfUnit = 4;  // stages of scale words per row read at once (32 bytes, one sector)
 constexpr int kOffSf = kStages * kStageBytes;
 constexpr int kSmem = kOffSf + kSfStages * kSfSlotBytes + 1024 /*barriers*/ + 1024 /*alignment*/;
 static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
@@ -88,7 +89,7 @@ enum : uint32_t {
 struct Bars {
   uint64_t full[kStages];     // TMA bytes of stage s landed
   uint64_t empty[kStages];    // the MMAs that read stage s (codes and scale columns) completed
-  uint64_t sf_full[kSfStages];   // scale slot j filled (one arrive per scale thread)
+  uint64_t sf_full[kSfStages];   // scale slot j filled (one arrive per scale warp)
   uint64_t sf_empty[kSfStages];  // the copies out of scale slot j completed
   uint64_t d_full;            // accumulator of the tile complete
   uint64_t d_empty;           // accumulator read out (one arrive per epilogue warp)
@@ -271,7 +272,7 @@ mxgemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
       mbar_init(&bars->empty[s], 1);
     }
     for (int j = 0; j < kSfStages; ++j) {
-      mbar_init(&bars->sf_full[j], 128);
+      mbar_init(&bars->sf_full[j], 4);
       mbar_init(&bars->sf_empty[j], 1);
     }
     mbar_init(&bars->d_full, 1);
@@ -392,19 +393,21 @@ mxgemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
     }
     __syncwarp();
   } else if (warp >= kWarpSf0 && warp < kWarpSf0 + 4) {
-    // thread st carries row st of the A tile and rows st, 128 + st of the W tile: row 32c + l
-    // of an operand goes to row l, bytes 4c .. 4c + 3, of its block
+    // thread st carries row 32c + l of the A tile and rows 32c + l, 128 + 32c + l of the W
+    // tile (c = st % 4, l = st / 4), each going to row l, bytes 4c .. 4c + 3, of its block:
+    // a warp's stores cover 128 contiguous bytes
     const int st = threadIdx.x - kWarpSf0 * 32;
-    const uint32_t off = uint32_t(16 * (st & 31) + 4 * (st >> 5));
+    const int rr = 32 * (st & 3) + (st >> 2);
+    const uint32_t off = uint32_t(16 * (st >> 2) + 4 * (st & 3));
     const uint8_t* bases[3] = {p.a_scales, p.w_scales, p.w_scales};
     const int64_t lim[3] = {p.T, p.O, p.O};
     auto tile_row = [&](int i, int r) {
       const int tile = int(blockIdx.x) + i * int(gridDim.x);
-      return r == 0 ? int64_t(tile / p.tiles_n) * kBM + st : int64_t(tile % p.tiles_n) * kBN + 128 * (r - 1) + st;
+      return r == 0 ? int64_t(tile / p.tiles_n) * kBM + rr : int64_t(tile % p.tiles_n) * kBN + 128 * (r - 1) + rr;
     };
     bool ok = true;
     // one stage's words (groups 0-3 and 4-7 of the stage for the three rows) into scale slot
-    // j; the writer fences its stores for the async proxy, then arrives
+    // j; every writer fences its stores for the async proxy, then one lane per warp arrives
     auto put = [&](int it, const uint32_t (&w)[3][2]) {
       const int j = it % kSfStages;
       if (it >= kSfStages &&
@@ -422,34 +425,44 @@ mxgemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
                        : "memory");
         }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive(&bars->sf_full[j]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->sf_full[j]);
     };
     if (p.sf_vec) {
-      // 16 bytes of a row (the groups of two stages) per load, issued two units ahead of use;
-      // unit n = stages 2v, 2v + 1 of local tile n / upt (v = n % upt)
-      const int upt = (p.nk + 1) / 2;
+      // kSfUnit stages (8 kSfUnit bytes of a row) per load unit, issued two units ahead of
+      // use; unit n = stages kSfUnit v .. kSfUnit v + kSfUnit - 1 of local tile n / upt
+      // (v = n % upt); 16-byte pieces past the row's end read as 0
+      constexpr int kQ = kSfUnit / 2;  // 16-byte pieces per row and unit
+      const int upt = (p.nk + kSfUnit - 1) / kSfUnit;
       const int n_units = n_local * upt;
-      auto load = [&](int n, uint4 (&b)[3]) {
+      auto load = [&](int n, uint4 (&b)[3][kQ]) {
         if (n >= n_units) return;
         const int i = n / upt;
-        const int64_t g0 = int64_t(n - i * upt) * 16;
+        const int64_t g0 = int64_t(n - i * upt) * (8 * kSfUnit);
 #pragma unroll
         for (int r = 0; r < 3; ++r) {
           const int64_t row = tile_row(i, r);
-          b[r] = row < lim[r] ? __ldg(reinterpret_cast<const uint4*>(bases[r] + row * p.sf_stride + g0))
-                              : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+          for (int q = 0; q < kQ; ++q)
+            b[r][q] = row < lim[r] && g0 + 16 * (q + 1) <= p.sf_stride
+                          ? __ldg(reinterpret_cast<const uint4*>(bases[r] + row * p.sf_stride + g0 + 16 * q))
+                          : make_uint4(0u, 0u, 0u, 0u);
         }
       };
-      auto store = [&](int n, const uint4 (&b)[3]) {
+      auto store = [&](int n, const uint4 (&b)[3][kQ]) {
         const int i = n / upt, v = n - i * upt;
-        const uint32_t w0[3][2] = {{b[0].x, b[0].y}, {b[1].x, b[1].y}, {b[2].x, b[2].y}};
-        put(i * p.nk + 2 * v, w0);
-        if (ok && 2 * v + 1 < p.nk) {
-          const uint32_t w1[3][2] = {{b[0].z, b[0].w}, {b[1].z, b[1].w}, {b[2].z, b[2].w}};
-          put(i * p.nk + 2 * v + 1, w1);
+#pragma unroll
+        for (int q = 0; q < kQ; ++q) {
+          const int kb = kSfUnit * v + 2 * q;
+          if (!ok || kb >= p.nk) return;
+          const uint32_t w0[3][2] = {{b[0][q].x, b[0][q].y}, {b[1][q].x, b[1][q].y}, {b[2][q].x, b[2][q].y}};
+          put(i * p.nk + kb, w0);
+          if (!ok || kb + 1 >= p.nk) return;
+          const uint32_t w1[3][2] = {{b[0][q].z, b[0][q].w}, {b[1][q].z, b[1][q].w}, {b[2][q].z, b[2][q].w}};
+          put(i * p.nk + kb + 1, w1);
         }
       };
-      uint4 b0[3], b1[3];
+      uint4 b0[3][kQ], b1[3][kQ];
       load(0, b0);
       load(1, b1);
       for (int n = 0; ok && n < n_units; n += 2) {

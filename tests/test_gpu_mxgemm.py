@@ -72,8 +72,10 @@ def _check(C, ref, bound, L):
     return float((err / tol).max())
 
 
+# L = 32, 96, 320: scale rows of 2, 4, 10 bytes (read word by word); 1536, 2560: rows of 48
+# and 80 bytes, whose last 16-byte piece of a wide read lies past the row
 SHAPES = [(300, 520, 8192), (129, 257, 14336), (1, 1, 32), (5, 3, 96), (77, 300, 320),
-          (256, 512, 4096), (130, 17, 2048)]
+          (256, 512, 4096), (130, 17, 2048), (70, 260, 1536), (33, 40, 2560)]
 
 
 @pytest.mark.parametrize("T,O,L", SHAPES, ids=[f"{t}x{o}x{l}" for t, o, l in SHAPES])
