@@ -29,7 +29,8 @@
 //   warp 16     TMA producer: x tiles (128 rows x N, 128B-swizzled) into a 3- or 4-stage ring
 //   warp 17     MMA issuer of stage A (A = BD(P1) in TMEM, or in SMEM when N = 128; B = x
 //               tile, MN-major); it also owns the TMEM allocation
-//   warp 18     MMA issuer of stage B (A = hi/lo Y in TMEM, B = P2^T in SMEM)
+//   warp 18     MMA issuer of stage B (A = hi/lo Y in TMEM, B = P2^T in SMEM); at
+//   warp 19     N = 96 and 112, warps 18 and 19 take the even and the odd local tiles
 //   warp 19     idle after the prologue
 // TMEM holds D_A slots (Y, then its hi / lo) and D_B slots (X''), two of each for N >= 96,
 // so stage A of the next tile runs while an epilogue group still encodes this one.
@@ -57,7 +58,7 @@ constexpr int kThreads = 640;  // five warpgroups
 // launched with, so setmaxnreg.inc always finds what it asks for.
 constexpr int kEpi = 4;  // epilogue warpgroups (warps 0-15)
 constexpr int kLaunchRegs = 96, kEpiRegs = 104, kLowRegs = 56;
-constexpr int kWarpProducer = 16, kWarpMmaA = 17, kWarpMmaB = 18;
+constexpr int kWarpProducer = 16, kWarpMmaA = 17, kWarpMmaB = 18, kWarpMmaB2 = 19;
 static_assert(128 * (kEpi * kEpiRegs + kLowRegs) <= kThreads * kLaunchRegs, "register split");
 constexpr uint64_t kTimeoutNs = 4000000000ull;  // 4 s: far beyond any legitimate wait (default)
 
@@ -101,6 +102,14 @@ struct Geo {
   static constexpr int kBlocks = N / 16;          // 16-column blocks of a row
   static constexpr int kGroups = (kBlocks + 1) / 2;  // published two blocks at a time
   static constexpr uint32_t kTmemCols = (!kP1Tmem && (kNA + kNB) * N <= 256) ? 256u : 512u;
+  // stage-B issuer warps: two (18 and 19, even and odd local tiles) where issuing a tile's
+  // 2N/16 MMAs and its barrier operations keeps one warp busy for the whole tile (N = 96,
+  // 112). Both slot counts must then be even, so that every slot's barriers are waited for
+  // by one of the two warps only: with an odd count one warp could reach tile b + kNA
+  // while the other has not yet been given tile b, and its parity wait would pass two
+  // phases early. One warp at N = 64 (no gain measured) and N = 128 (measured slower).
+  static constexpr int kBIss = (N == 96 || N == 112) ? 2 : 1;
+  static_assert(kBIss == 1 || (kNA % 2 == 0 && kNB % 2 == 0), "two stage-B warps need even slot counts");
 };
 
 struct Bars {
@@ -112,7 +121,7 @@ struct Bars {
   uint64_t ys_full[4][4];   // D_A slot: hi / lo of column group g (two 16-column blocks) written
   uint64_t da_free[4];      // D_A slot: stage B that read it has completed
   uint64_t tm_empty[4];     // D_B slot: X'' read out by the epilogue
-  uint64_t mma_done[2];
+  uint64_t mma_done[3];
   uint32_t tmem_base;
   int abort;
   uint64_t timeout_ns;  // limit of every bounded wait of this launch
@@ -140,18 +149,17 @@ __device__ __forceinline__ uint64_t globaltimer() {
 __device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
 }
-// Waits for a phase to complete, with the thread suspended in hardware until it does or
-// kSuspendNs pass (a short hint would make waiting warps spin, taking issue slots from the
-// warps that work on their sub-partition).
-constexpr uint32_t kSuspendNs = 1000000;
+// Waits for a phase to complete, the thread suspended in hardware until it does or a
+// limit the hardware chooses passes. (An explicit suspend-time hint of 1 ms or of 2-20 us
+// measured 1-4 % slower over the whole kernel: the waiters woke later.)
 __device__ __forceinline__ bool mbar_try_wait(uint32_t b, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(b), "r"(parity), "n"(kSuspendNs)
+      : "r"(b), "r"(parity)
       : "memory");
   return ok != 0;
 }
@@ -494,6 +502,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     }
     mbar_init(&bars->mma_done[0], 1);
     mbar_init(&bars->mma_done[1], 1);
+    mbar_init(&bars->mma_done[2], 1);
     bars->abort = 0;
     bars->timeout_ns = p.timeout_ns != 0 ? p.timeout_ns : kTimeoutNs;
     for (int g = 0; g < kEpi; ++g) bars->group_exit[g][0] = bars->group_exit[g][1] = 0;
@@ -619,20 +628,22 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
         }
       }
     }
-  } else if (warp == kWarpMmaA || warp == kWarpMmaB) {
+  } else if (warp == kWarpMmaA || warp == kWarpMmaB || (G::kBIss == 2 && warp == kWarpMmaB2)) {
     // ---------------- MMA issuers ----------------
-    // Warp 17 issues stage A of every tile, warp 18 stage B, each in tile order and each
-    // with blocking waits (a waiting warp takes no issue slots from the epilogue warps on
-    // its sub-partition). The whole warp runs the loop, so descriptors stay warp-uniform,
-    // and one elected lane issues.
+    // Warp 17 issues stage A of every tile in tile order; stage B is issued by warp 18, or
+    // by warps 18 and 19 taking every other tile (kBIss), each in its own tile order; all
+    // with blocking waits. The whole warp runs the loop, so descriptors stay warp-uniform,
+    // and one elected lane issues; each warp commits only its own MMAs.
     //   stage A of tile a: x tile landed; D_A slot free (stage B of tile a - kNA done).
     //   stage B of tile b: D_B slot free (tile b - kNB read out); then each pair of
     //                      16-column blocks of hi / lo as soon as it is published.
-    // Every barrier has one waiter that takes its phases in order. A waiter is never two
+    // Every barrier has one waiter that takes its phases in order, and none is ever two
     // phases behind: stage A of tile i + kEpi waits for stage B of tile i + kEpi - kNA,
-    // issued after stage B of tile i (kNA <= kEpi), which waits for the split of tile i;
-    // stage B of tile i + kEpi is issued after stage B of tile i + kNB (kNB <= kEpi), which
-    // waits for the epilogue to read tile i out.
+    // which waits for the split of tile i + kEpi - kNA, issued after that of tile i; a
+    // stage-B warp waits for the split of tile b (phase b / kNA of a D_A slot) and for the
+    // read-out of tile b - kNB, and the next phase of either barrier needs stage B of tile
+    // b itself. With two stage-B warps both slot counts are even, so the tiles of a slot
+    // all belong to one of them.
     setmaxnreg_dec<kLowRegs>();
     const int n_local = (blockIdx.x < num_tiles) ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     const int mb = warp - kWarpMmaA;
@@ -662,7 +673,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       constexpr uint32_t kIdB = idesc_f16(false, false, false, N);
       const uint64_t p2_desc = desc64(sbase + G::kOffP2, 16);
       bool ok = true;
-      for (int b = 0; ok && b < n_local; ++b) {
+      for (int b = mb - 1; ok && b < n_local; b += G::kBIss) {
         const int sa = b % G::kNA;
         if (b >= G::kNB &&
             !warp_wait(&bars->tm_empty[b % G::kNB], ((b / G::kNB) - 1) & 1, bars, p.status, kStMmaTmemEmpty))
@@ -695,8 +706,8 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
       }
     }
     __syncwarp();
-  } else if (warp == kWarpMmaB + 1) {
-    setmaxnreg_dec<kLowRegs>();  // idle warp of the producer / MMA warpgroup
+  } else if (warp == kWarpMmaB2) {
+    setmaxnreg_dec<kLowRegs>();  // idle warp of the producer / MMA warpgroup (N = 128)
   } else {
     // ---------------- epilogue warpgroups: split, then quantize, the same tile ----------------
     // Group eg takes the local tiles i = eg (mod kEpi). For its tile it first splits Y

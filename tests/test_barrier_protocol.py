@@ -4,8 +4,8 @@ This is a host-side check of a design argument, not a test of the CUDA code: the
 restates, by hand, the waits, arrivals and MMA commits of the roles in
 `rotation_bit_quantization_token_b200/csrc/fq_tc.cu` for one CTA:
 - the TMA producer;
-- the stage-A and stage-B MMA issuers, whose MMAs and commits complete asynchronously but
-  in issue order;
+- the stage-A MMA issuer and one or two stage-B MMA issuers (two take the even and the odd
+  tiles), whose MMAs and commits complete asynchronously, each issuer's in its issue order;
 - four epilogue groups of four warps each, every warp its own actor.
 
 mbarriers follow their parity semantics: a wait for parity P passes while the barrier's
@@ -20,7 +20,9 @@ ever two phases behind.
 Planted mistakes must each be caught, which shows the model can fail:
 - stage B's release of a Y slot left out;
 - a parity off by one;
-- an X'' slot reused without its wait.
+- an X'' slot reused without its wait;
+- with two stage-B issuers, one that waits for the read-out of its own previous tile on the
+  slot instead of tile b - kNB.
 """
 
 import random
@@ -44,9 +46,10 @@ class _Bar:
             self.done += 1
 
 
-def run_protocol(T, kNA, kNB, kStages, kGroups, seed, kEpi=4, plant=None):
+def run_protocol(T, kNA, kNB, kStages, kGroups, seed, kEpi=4, plant=None, kBIss=1):
     """One CTA over T local tiles. kNA / kNB: TMEM slots of Y and X''; kGroups: pairs of
-    16-column blocks per row. Returns the number of scheduler steps; raises Viol."""
+    16-column blocks per row; kBIss: stage-B issuers. Returns the number of scheduler steps;
+    raises Viol."""
     rng = random.Random(seed)
     bars = {}
 
@@ -96,11 +99,17 @@ def run_protocol(T, kNA, kNB, kStages, kGroups, seed, kEpi=4, plant=None):
             yield ("commit", "A", ("x_empty", s))
             yield ("commit", "A", ("da_full", a % kEpi))
 
-    def stage_b():
-        for b in range(T):
+    def stage_b(r):
+        iss = "B%d" % r
+        for b in range(r, T, kBIss):
             sa, sb = b % kNA, b % kNB
             if b >= kNB and plant != "no tm_empty wait":
-                yield ("wait", ("tm_empty", sb), ((b // kNB) - 1) & 1, (b // kNB) - 1)
+                # the read-out of tile b - kNB (the planted mistake: of this issuer's own
+                # previous tile on the slot, kBIss * kNB back)
+                back = kNB * kBIss if plant == "own previous tile" else kNB
+                if b >= back:
+                    k = (b - back) // kNB
+                    yield ("wait", ("tm_empty", sb), k & 1, k)
             for g in range(kGroups):
                 yield ("wait", ("ys_full", sa, g), (b // kNA) & 1, b // kNA)
 
@@ -108,10 +117,10 @@ def run_protocol(T, kNA, kNB, kStages, kGroups, seed, kEpi=4, plant=None):
                     for q in range(4):
                         check(("HL", sa, g, q), b)
                         mem[("D", sb, q)] = (b, g)
-                yield ("mma", "B", mma)
-            yield ("commit", "B", ("db_full", b % kEpi))
+                yield ("mma", iss, mma)
+            yield ("commit", iss, ("db_full", b % kEpi))
             if plant != "da_free before stage B":
-                yield ("commit", "B", ("da_free", sa))
+                yield ("commit", iss, ("da_free", sa))
 
     def epilogue_warp(eg, q):
         jj = 0
@@ -132,12 +141,15 @@ def run_protocol(T, kNA, kNB, kStages, kGroups, seed, kEpi=4, plant=None):
             yield ("arrive", ("tm_empty", sb))
             jj += 1
 
-    actors = {"producer": producer(), "A": stage_a(), "B": stage_b()}
+    actors = {"producer": producer(), "A": stage_a()}
+    for r in range(kBIss):
+        actors["B%d" % r] = stage_b(r)
     for eg in range(kEpi):
         for q in range(4):
             actors[("epilogue", eg, q)] = epilogue_warp(eg, q)
     cur = dict.fromkeys(actors)
-    queues = {"A": [], "B": []}
+    queues = {"A": []}
+    queues.update({"B%d" % r: [] for r in range(kBIss)})
     landing = []
     finished = set()
     steps = 0
@@ -167,7 +179,7 @@ def run_protocol(T, kNA, kNB, kStages, kGroups, seed, kEpi=4, plant=None):
             # re-draw every actor's speed now and then, so that some actor stalls for a
             # while and others run ahead (the orders a uniform choice almost never makes)
             speed = {c: rng.choice((0.01, 0.1, 1.0, 1.0, 4.0)) for c in
-                     list(actors) + ["q:A", "q:B", "tma"]}
+                     list(actors) + ["q:" + q for q in queues] + ["tma"]}
         weights = [speed[c[1] if c[0] == "actor" else ("q:" + c[1] if c[0] == "mma" else "tma")]
                    for c in choices]
         kind, k = rng.choices(choices, weights)[0]
@@ -197,24 +209,53 @@ def run_protocol(T, kNA, kNB, kStages, kGroups, seed, kEpi=4, plant=None):
             bars[("x_full", s)].arrive()
 
 
-# (N, kNA, kNB, kStages, pairs per row) of the kernel's geometry for each N it covers
-SHAPES = [(64, 4, 3, 4, 2), (80, 3, 2, 4, 3), (96, 2, 2, 4, 3), (112, 2, 2, 4, 4), (128, 2, 2, 3, 4)]
+# (N, kNA, kNB, kStages, pairs per row, stage-B issuers) of the kernel's geometry for each N
+# it covers
+SHAPES = [(64, 4, 3, 4, 2, 1), (80, 3, 2, 4, 3, 1), (96, 2, 2, 4, 3, 2), (112, 2, 2, 4, 4, 2),
+          (128, 2, 2, 3, 4, 1)]
 
 
-@pytest.mark.parametrize("N,kNA,kNB,kStages,pairs", SHAPES)
-def test_protocol_has_no_deadlock_phase_slip_or_stale_read(N, kNA, kNB, kStages, pairs):
+@pytest.mark.parametrize("N,kNA,kNB,kStages,pairs,kBIss", SHAPES)
+def test_protocol_has_no_deadlock_phase_slip_or_stale_read(N, kNA, kNB, kStages, pairs, kBIss):
     for T in (1, 2, 3, 5, 9, 17):
         for seed in range(60):
-            run_protocol(T, kNA, kNB, kStages, pairs, seed)
+            run_protocol(T, kNA, kNB, kStages, pairs, seed, kBIss=kBIss)
 
 
-@pytest.mark.parametrize("plant", ["da_free before stage B", "da_free parity", "no tm_empty wait"])
+@pytest.mark.parametrize("N,kNA,kNB,kStages,pairs", [(96, 2, 2, 4, 3), (112, 2, 2, 4, 4), (128, 2, 2, 3, 4)])
+def test_protocol_with_the_other_issuer_count(N, kNA, kNB, kStages, pairs):
+    """One and two stage-B issuers where both slot counts are even (either is a valid build)."""
+    for kBIss in (1, 2):
+        for T in (2, 5, 9, 17):
+            for seed in range(30):
+                run_protocol(T, kNA, kNB, kStages, pairs, seed, kBIss=kBIss)
+
+
+def test_two_issuers_with_an_odd_slot_count_are_caught():
+    """Why the kernel takes two stage-B warps only with even slot counts: at N = 80 (three
+    D_A slots) one warp can wait for the split of tile b + 3 before tile b was split, and
+    its parity wait passes two phases early."""
+    caught = False
+    for T in (9, 17):
+        for seed in range(400):
+            try:
+                run_protocol(T, 3, 2, 4, 3, seed, kBIss=2)
+            except Viol:
+                caught = True
+                break
+        if caught:
+            break
+    assert caught
+
+
+@pytest.mark.parametrize("plant", ["da_free before stage B", "da_free parity", "no tm_empty wait",
+                                   "own previous tile"])
 def test_planted_protocol_mistakes_are_caught(plant):
     caught = False
     for T in (3, 5, 9, 17):
         for seed in range(200):
             try:
-                run_protocol(T, 2, 2, 4, 4, seed, plant=plant)
+                run_protocol(T, 2, 2, 4, 4, seed, plant=plant, kBIss=2)
             except Viol:
                 caught = True
                 break
