@@ -41,7 +41,7 @@ CSRC = os.path.join(ROOT, "rotation_bit_quantization_token_b200", "csrc")
 def parse_args(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default=BENCH_WORKLOAD, choices=sorted(WORKLOADS))
@@ -305,10 +305,12 @@ def run_reference(args, rank, world):
     if rank != 0:
         return 0
     # each step times the oracle on the same bounded sample of the workload; the sample
-    # size is fixed by a sizing run before the warm-up, so every step does the same work
+    # size is fixed by a sizing run before the warm-up, so every step does the same work,
+    # about 2 s of it, less when many steps are asked for (the run stays near two minutes)
     import oracle
     from threadpoolctl import threadpool_info
-    _, n_tok, _, threads = bounded_oracle_sample(w, seed=0, target_s=2.0)
+    target_s = min(2.0, 120.0 / max(1, args.steps + args.warmup))
+    _, n_tok, _, threads = bounded_oracle_sample(w, seed=0, target_s=target_s)
     x, P1, P2 = make_inputs(w.with_tokens(n_tok), seed=0)
     xf = x.float().numpy().astype(np.float64)
     p1 = P1.float().numpy().astype(np.float64)
@@ -342,6 +344,7 @@ def run_reference(args, rank, world):
                    "step": f"the oracle over {n_tok} of the workload's {w.K} tokens"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "nproc": logical, "usable_cores": usable,
+                         "omp_num_threads": os.environ.get("OMP_NUM_THREADS"),
                          "sample": f"{n_tok} tokens of {w.name} per step "
                                    f"({ms_per_step / 1e3:.2f} s each), rate in tokens/s"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -393,6 +396,7 @@ def run_ours(args, rank, world, local):
         cpu = {"value": r, "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": f"{n} tokens of {w.name} ({dt:.1f} s), scaled to tokens/s",
                "nproc": logical, "usable_cores": usable,
+               "omp_num_threads": os.environ.get("OMP_NUM_THREADS"),
                "single_core": {"value": r1, "unit": UNIT,
                                "sample": f"{n1} tokens on one BLAS thread ({dt1:.1f} s)"}}
 
@@ -464,7 +468,7 @@ def run_ours(args, rank, world, local):
         dist.barrier()
     clock_info = clocks.stop() if clocks else None
     elapsed_ms = t_start.elapsed_time(t_end)
-    kernel_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    kernel_ms = float(np.median([a.elapsed_time(b) for a, b in evs]))  # per-launch median
     elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
     kernel_ms_max = max_over_ranks(kernel_ms, world, dev)
     status = fq.device_status()
