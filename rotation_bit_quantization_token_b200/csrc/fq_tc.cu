@@ -478,11 +478,56 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
   const int num_tiles = int((rows_total + 127) / 128);
 
   // ---- prologue: P2 scale, BD(P1) and P2^T operands, barriers, TMEM ----
+  // TMEM first, so that BD(P1) can go there right after the first barrier. Every global
+  // read of P1 and P2 is then issued at once (one round trip), into one register buffer
+  // whatever the thread's part: threads 256 .. 256 + (N/8)^2 - 1 each hold an 8 x 8 block
+  // of P2 (whose maximum is taken from the same registers); threads 128 .. 255 a row of
+  // BD(P1) for TMEM (warps 4-7: each row's TMEM lane lies in its warp's lane quarter);
+  // threads 0 .. 255 store the chunks of BD(P1)'s shared-memory form as they arrive.
+  if (warp == kWarpMmaA) tmem_alloc(&bars->tmem_base, G::kTmemCols);
+  constexpr int NB = N / 8;
+  static_assert(256 + NB * NB <= kThreads, "one P2 block per thread");
+  const int pb = tid - 256;
+  const bool has_pb = pb >= 0 && pb < NB * NB;
+  const bool has_p1row = G::kP1Tmem && tid >= 128 && tid < 256;
+  uint4 buf[16];
+  if (has_pb && p.P2 != nullptr) {
+    const int jb = pb / NB, nb = pb % NB;
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj)
+      buf[jj] = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.P2) + (jb * 8 + jj) * N + nb * 8);
+  } else if (has_p1row) {
+    const int r = tid - 128;
+#pragma unroll
+    for (int kc = 0; kc < 16; ++kc) {
+      const int k = kc * 8;
+      buf[kc] = r / M == k / M
+                    ? *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.P1) + (r % M) * M + (k % M))
+                    : make_uint4(0u, 0u, 0u, 0u);
+    }
+  } else if (!G::kP1Tmem && tid < 256) {
+    // BD(P1): 128 x 128, K-major, 128B swizzle; element (r, k) = P1[r % M][k % M] on the
+    // diagonal blocks (r / M == k / M), else 0.
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int c = tid + 256 * q;
+      const int r = c >> 4, kc = c & 15, k = kc * 8;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (r / M == k / M)
+        v = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.P1) + (r % M) * M + (k % M));
+      const uint32_t off = G::kOffP1 + (kc >> 3) * 16384 + r * 128 + ((((kc & 7) ^ (r & 7))) << 4);
+      *reinterpret_cast<uint4*>(smem + off) = v;
+    }
+  }
   float lmax = 0.0f;
-  if (p.P2 != nullptr) {
-    for (int i = tid; i < N * N; i += kThreads) lmax = fmaxf(lmax, fabsf(ld16f<kF16>(p.P2, i)));
-  } else {
-    lmax = 1.0f;
+  if (has_pb && p.P2 != nullptr) {
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      float f[8];
+      unpack8<kF16>(buf[jj], f);
+#pragma unroll
+      for (int nn = 0; nn < 8; ++nn) lmax = fmaxf(lmax, fabsf(f[nn]));
+    }
   }
   lmax = warp_max(lmax);
   if (lane == 0) bars->wmax[warp] = lmax;
@@ -508,7 +553,18 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     for (int g = 0; g < kEpi; ++g) bars->group_exit[g][0] = bars->group_exit[g][1] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  if (has_p1row) {
+    // BD(P1) into TMEM as the A operand of stage A: lane r holds row r, column c the
+    // elements (r, 2c) and (r, 2c + 1) in its low and high halves
+    const uint32_t t_row = tmem + (uint32_t((warp & 3) * 32) << 16) + G::kP1Col;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tmem_st16(t_row + 16 * j, reinterpret_cast<const uint32_t*>(buf + 4 * j));
+    tmem_wait_st();
+  }
   // the producer issues its first round of x loads now: nothing below writes the x ring, so
   // their latency overlaps the rest of the prologue (a small launch spends a good part of its
   // time there)
@@ -525,30 +581,19 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
   float p2max = 0.0f;
 #pragma unroll
   for (int w = 0; w < kThreads / 32; ++w) p2max = fmaxf(p2max, bars->wmax[w]);
+  if (p.P2 == nullptr) p2max = 1.0f;  // P2 skipped: the identity
   const int t_exp = prescale_exp(p2max);
   const float p2scale = exp2i(t_exp);
 
-  // BD(P1): 128 x 128, K-major, 128B swizzle; element (r, k) = P1[r % M][k % M] on the
-  // diagonal blocks (r / M == k / M), else 0.
-  for (int c = tid; !G::kP1Tmem && c < 128 * 16; c += kThreads) {
-    const int r = c >> 4, kc = c & 15, k = kc * 8;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (r / M == k / M)
-      v = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.P1) + (r % M) * M + (k % M));
-    const uint32_t off = G::kOffP1 + (kc >> 3) * 16384 + r * 128 + ((((kc & 7) ^ (r & 7))) << 4);
-    *reinterpret_cast<uint4*>(smem + off) = v;
-  }
   // P2^T scaled by 2^t as fp16: N rows (n), K = N (j), K-major, 128B swizzle.
-  constexpr int NB = N / 8;
-  for (int blk = tid; blk < NB * NB; blk += kThreads) {
-    const int jb = blk / NB, nb = blk % NB;
+  if (has_pb) {
+    const int jb = pb / NB, nb = pb % NB;
     float v[8][8];
 #pragma unroll
     for (int jj = 0; jj < 8; ++jj) {
       const int j = jb * 8 + jj;
       if (p.P2 != nullptr) {
-        const uint4 q = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.P2) + j * N + nb * 8);
-        unpack8<kF16>(q, v[jj]);
+        unpack8<kF16>(buf[jj], v[jj]);
       } else {
 #pragma unroll
         for (int nn = 0; nn < 8; ++nn) v[jj][nn] = (j == nb * 8 + nn) ? 1.0f : 0.0f;
@@ -566,37 +611,9 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     }
   }
   fence_proxy_async();
-  if (warp == kWarpMmaA) tmem_alloc(&bars->tmem_base, G::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = bars->tmem_base;
-  if constexpr (G::kP1Tmem) {
-    // BD(P1) into TMEM as the A operand of stage A: lane r holds row r, column c the
-    // elements (r, 2c) and (r, 2c + 1) in its low and high halves
-    if (tid < 128) {
-      const int r = tid;
-      uint32_t w[64];
-#pragma unroll
-      for (int kc = 0; kc < 16; ++kc) {
-        const int k = kc * 8;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (r / M == k / M)
-          v = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.P1) + (r % M) * M + (k % M));
-        w[4 * kc] = v.x;
-        w[4 * kc + 1] = v.y;
-        w[4 * kc + 2] = v.z;
-        w[4 * kc + 3] = v.w;
-      }
-      const uint32_t t_row = tmem + (uint32_t(warp * 32) << 16) + G::kP1Col;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) tmem_st16(t_row + 16 * j, w + 16 * j);
-      tmem_wait_st();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-  }
 
   if (warp == kWarpProducer) {
     // ---------------- TMA producer ----------------
