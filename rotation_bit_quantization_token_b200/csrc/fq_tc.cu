@@ -485,6 +485,43 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
   // BD(P1) for TMEM (warps 4-7: each row's TMEM lane lies in its warp's lane quarter);
   // threads 0 .. 255 store the chunks of BD(P1)'s shared-memory form as they arrive.
   if (warp == kWarpMmaA) tmem_alloc(&bars->tmem_base, G::kTmemCols);
+  // The producer thread initializes the barriers and at once issues its first round of x
+  // loads: nothing in the prologue writes the x ring, so their latency overlaps all of it
+  // (a small launch spends a good part of its time there). The other threads use the
+  // barriers only after the first __syncthreads.
+  const int n_early = (warp == kWarpProducer && lane == 0 && !p.stall_loads && int(blockIdx.x) < num_tiles)
+                          ? min((num_tiles - 1 - int(blockIdx.x)) / int(gridDim.x) + 1, G::kStages)
+                          : 0;
+  if (warp == kWarpProducer && lane == 0) {
+    for (int s = 0; s < G::kStages; ++s) {
+      mbar_init(&bars->x_full[s], 1);
+      mbar_init(&bars->x_empty[s], 1);
+    }
+    for (int a = 0; a < 4; ++a) {
+      for (int g = 0; g < 4; ++g) mbar_init(&bars->ys_full[a][g], 4);
+      mbar_init(&bars->da_free[a], 1);
+      mbar_init(&bars->tm_empty[a], 4);
+    }
+    for (int g = 0; g < kEpi; ++g) {
+      mbar_init(&bars->da_full[g], 1);
+      mbar_init(&bars->db_full[g], 1);
+    }
+    mbar_init(&bars->mma_done[0], 1);
+    mbar_init(&bars->mma_done[1], 1);
+    mbar_init(&bars->mma_done[2], 1);
+    bars->abort = 0;
+    bars->timeout_ns = p.timeout_ns != 0 ? p.timeout_ns : kTimeoutNs;
+    for (int g = 0; g < kEpi; ++g) bars->group_exit[g][0] = bars->group_exit[g][1] = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    fence_proxy_async();  // the initialized barriers, before the bulk copies that complete on them
+    for (int i = 0; i < n_early; ++i) {
+      mbar_arrive_expect_tx(&bars->x_full[i], G::kXStage);
+#pragma unroll
+      for (int a = 0; a < G::kAtoms; ++a)
+        tma_load_2d(sbase + G::kOffX + i * G::kXStage + a * 16384, &tmap, a * 64,
+                    (int(blockIdx.x) + i * int(gridDim.x)) * 128, &bars->x_full[i]);
+    }
+  }
   constexpr int NB = N / 8;
   static_assert(256 + NB * NB <= kThreads, "one P2 block per thread");
   const int pb = tid - 256;
@@ -531,28 +568,6 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
   }
   lmax = warp_max(lmax);
   if (lane == 0) bars->wmax[warp] = lmax;
-  if (tid == 0) {
-    for (int s = 0; s < G::kStages; ++s) {
-      mbar_init(&bars->x_full[s], 1);
-      mbar_init(&bars->x_empty[s], 1);
-    }
-    for (int a = 0; a < 4; ++a) {
-      for (int g = 0; g < 4; ++g) mbar_init(&bars->ys_full[a][g], 4);
-      mbar_init(&bars->da_free[a], 1);
-      mbar_init(&bars->tm_empty[a], 4);
-    }
-    for (int g = 0; g < kEpi; ++g) {
-      mbar_init(&bars->da_full[g], 1);
-      mbar_init(&bars->db_full[g], 1);
-    }
-    mbar_init(&bars->mma_done[0], 1);
-    mbar_init(&bars->mma_done[1], 1);
-    mbar_init(&bars->mma_done[2], 1);
-    bars->abort = 0;
-    bars->timeout_ns = p.timeout_ns != 0 ? p.timeout_ns : kTimeoutNs;
-    for (int g = 0; g < kEpi; ++g) bars->group_exit[g][0] = bars->group_exit[g][1] = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -564,19 +579,6 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) tmem_st16(t_row + 16 * j, reinterpret_cast<const uint32_t*>(buf + 4 * j));
     tmem_wait_st();
-  }
-  // the producer issues its first round of x loads now: nothing below writes the x ring, so
-  // their latency overlaps the rest of the prologue (a small launch spends a good part of its
-  // time there)
-  const int n_early = (warp == kWarpProducer && lane == 0 && !p.stall_loads && int(blockIdx.x) < num_tiles)
-                          ? min((num_tiles - 1 - int(blockIdx.x)) / int(gridDim.x) + 1, G::kStages)
-                          : 0;
-  for (int i = 0; i < n_early; ++i) {
-    mbar_arrive_expect_tx(&bars->x_full[i], G::kXStage);
-#pragma unroll
-    for (int a = 0; a < G::kAtoms; ++a)
-      tma_load_2d(sbase + G::kOffX + i * G::kXStage + a * 16384, &tmap, a * 64,
-                  (int(blockIdx.x) + i * int(gridDim.x)) * 128, &bars->x_full[i]);
   }
   float p2max = 0.0f;
 #pragma unroll
