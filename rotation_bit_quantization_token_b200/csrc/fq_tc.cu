@@ -26,7 +26,7 @@
 //               row of X'' (twice: block maxima, then the codes, so that a thread never
 //               holds a whole row), releases the buffer, forms per-token or per-group scales
 //               and codes, stages them in shared memory and stores them with bulk copies
-//   warp 16     TMA producer: x tiles (128 rows x N, 128B-swizzled) into a 3- or 4-stage ring
+//   warp 16     TMA producer: x tiles (128 rows x N, 128B-swizzled) into a 3- to 5-stage ring
 //   warp 17     MMA issuer of stage A (A = BD(P1) in TMEM, or in SMEM when N = 128; B = x
 //               tile, MN-major); it also owns the TMEM allocation
 //   warp 18     MMA issuer of stage B (A = hi/lo Y in TMEM, B = P2^T in SMEM); at
@@ -51,7 +51,7 @@
 namespace fq {
 namespace {
 
-constexpr int kStagesMax = 4;
+constexpr int kStagesMax = 5;
 constexpr int kThreads = 640;  // five warpgroups
 // Register split (setmaxnreg): launched at kLaunchRegs per thread; the four epilogue
 // warpgroups rise to kEpiRegs and the producer / MMA warpgroup drops to kLowRegs. The shares add up to no more than the registers the block was
@@ -74,8 +74,10 @@ struct Geo {
   static_assert(N % 16 == 0 && N >= 64 && N <= 128, "tensor-core kernel covers N in [64,128], N % 16 == 0");
   static constexpr int kAtoms = (N + 63) / 64;              // 64-element swizzle atoms along N
   static constexpr int kXStage = kAtoms * 128 * 128;        // bytes per x stage
-  // x ring depth: four stages, three at N = 128 where BD(P1) stays in shared memory
-  static constexpr int kStages = N == 128 ? 3 : 4;
+  // x ring depth: five stages at N = 80 .. 112 (2-3 % faster than four at 128 x 112),
+  // four at N = 64 (eight measured slower: the longer first round of loads delays the
+  // first tile), three at N = 128 where BD(P1) stays in shared memory
+  static constexpr int kStages = N == 128 ? 3 : (N == 64 ? 4 : 5);
   // BD(P1) sits in TMEM (64 columns; stage A is then a TS MMA that reads only the x tile
   // from shared memory, 3.5 KB instead of 7.5 KB per MMA at N = 112) when four N-column
   // slots still fit beside it; otherwise in shared memory, 128 x 128, two K atoms (SS).

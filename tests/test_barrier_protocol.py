@@ -211,7 +211,7 @@ def run_protocol(T, kNA, kNB, kStages, kGroups, seed, kEpi=4, plant=None, kBIss=
 
 # (N, kNA, kNB, kStages, pairs per row, stage-B issuers) of the kernel's geometry for each N
 # it covers
-SHAPES = [(64, 4, 3, 4, 2, 1), (80, 3, 2, 4, 3, 1), (96, 2, 2, 4, 3, 2), (112, 2, 2, 4, 4, 2),
+SHAPES = [(64, 4, 3, 4, 2, 1), (80, 3, 2, 5, 3, 1), (96, 2, 2, 5, 3, 2), (112, 2, 2, 5, 4, 2),
           (128, 2, 2, 3, 4, 1)]
 
 
@@ -222,7 +222,7 @@ def test_protocol_has_no_deadlock_phase_slip_or_stale_read(N, kNA, kNB, kStages,
             run_protocol(T, kNA, kNB, kStages, pairs, seed, kBIss=kBIss)
 
 
-@pytest.mark.parametrize("N,kNA,kNB,kStages,pairs", [(96, 2, 2, 4, 3), (112, 2, 2, 4, 4), (128, 2, 2, 3, 4)])
+@pytest.mark.parametrize("N,kNA,kNB,kStages,pairs", [(96, 2, 2, 5, 3), (112, 2, 2, 5, 4), (128, 2, 2, 3, 4)])
 def test_protocol_with_the_other_issuer_count(N, kNA, kNB, kStages, pairs):
     """One and two stage-B issuers where both slot counts are even (either is a valid build)."""
     for kBIss in (1, 2):
