@@ -443,23 +443,21 @@ def run_ours(args, rank, world, local):
     if clocks:
         clocks.start()
         time.sleep(0.3)
-    # per-launch events on the launching stream: the step is one kernel launch. The timed
-    # launches queue up behind a short GPU sleep (outside the timed region), so that the
-    # host has enqueued them all before the first one runs: the events then time the
-    # device work, not the host's Python and ctypes time between calls, which is longer
-    # than the kernel of the smaller workloads. `queue_primed` records that the sleep was
-    # still running when the last launch had been enqueued.
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
+    # CUDA events on the launching stream at the two ends of the timed region; the step is
+    # one kernel launch, so the average launch duration is the region over the launches. The
+    # timed launches queue up behind a short GPU sleep (outside the timed region), so that
+    # the host has enqueued them all before the first one runs and they run back to back:
+    # the events then time the device work, not the host's Python and ctypes time between
+    # calls, which is longer than the kernel of the smaller workloads (events between the
+    # launches would add their own gaps, about 2 us a launch). `queue_primed` records that
+    # the sleep was still running when the last launch had been enqueued.
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     launches = 0
     torch.cuda._sleep(int(PRIME_CYCLES_PER_STEP * max(args.steps, 20)))
     t_start.record(stream)
     for i in range(args.steps):
-        evs[i][0].record(stream)
         step()
-        evs[i][1].record(stream)
         launches += fq.last_launch_count
     t_end.record(stream)
     queue_primed = not t_start.query()
@@ -468,7 +466,7 @@ def run_ours(args, rank, world, local):
         dist.barrier()
     clock_info = clocks.stop() if clocks else None
     elapsed_ms = t_start.elapsed_time(t_end)
-    kernel_ms = float(np.median([a.elapsed_time(b) for a, b in evs]))  # per-launch median
+    kernel_ms = elapsed_ms / max(launches, 1)  # average launch duration
     elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
     kernel_ms_max = max_over_ranks(kernel_ms, world, dev)
     status = fq.device_status()
