@@ -27,8 +27,10 @@ def _method_byte(amax, D):
     Eq, Mq = (qb >> 23) & 0xFF, qb & 0x7FFFFF
     common = (Eq >= 1) & (Eq <= 253) & (Mq >= 4) & (Mq <= 0x7FFFFA)
     k = np.where(Eq == 0, -126, np.where(Mq <= 3, Eq - 127, Eq - 126))
-    # S next to 2^-126: 0 (subnormal S), 1 (S = 2^-126) or 2, from terms scaled by 2^64
-    a64 = (a.astype(np.float64) * 2.0 ** 64).astype(np.float32)
+    # S next to 2^-126: 0 (subnormal S), 1 (S = 2^-126) or 2, from terms scaled by 2^64 (only
+    # used there: for large amax the scaled term overflows to inf and is not read)
+    with np.errstate(over="ignore"):
+        a64 = (a.astype(np.float64) * 2.0 ** 64).astype(np.float32)
     r0 = (a64.astype(np.float64) - np.float64(D32) * 2.0 ** -62).astype(np.float32)
     t0 = np.float32(np.float64(D32) * 2.0 ** -86)
     bottom = np.where(r0 > t0, 2, np.where(r0 >= -t0, 1, 0))
