@@ -248,15 +248,6 @@ __device__ __forceinline__ void mma_ss_e(uint32_t d, uint64_t a, uint64_t b, uin
       "l"(a), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
-__device__ __forceinline__ void mma_ts_e(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\t"
-      "elect.sync r|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
 // Stage B of one 16-column block: the hi MMA (A at a_hi, accumulate flag acc_first) then
 // the lo MMA (A 8 columns further, always accumulating), both with B = b_desc, under one
 // election: the issuing warp shares its sub-partition with busy epilogue warps, so every
