@@ -107,6 +107,17 @@ KERNEL_SOURCES = {
 PRIME_CYCLES_PER_STEP = 400_000
 
 
+def prime_stream(steps):
+    """Queues a GPU sleep on the current stream, so that the launches enqueued after it wait
+    until the host has enqueued them all (torch.cuda._sleep is torch's own spin kernel);
+    False where this torch has no such call (the timing then holds the host's gaps)."""
+    sleep = getattr(torch.cuda, "_sleep", None)
+    if sleep is None:
+        return False
+    sleep(int(PRIME_CYCLES_PER_STEP * max(steps, 20)))
+    return True
+
+
 def kernel_source_hash(kernel="tcgen05"):
     """Hash of the source files of one kernel (a recorded DRAM-traffic figure is valid only
     for the source it was captured on)."""
@@ -454,13 +465,13 @@ def run_ours(args, rank, world, local):
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     launches = 0
-    torch.cuda._sleep(int(PRIME_CYCLES_PER_STEP * max(args.steps, 20)))
+    primed = prime_stream(args.steps)
     t_start.record(stream)
     for i in range(args.steps):
         step()
         launches += fq.last_launch_count
     t_end.record(stream)
-    queue_primed = not t_start.query()
+    queue_primed = primed and not t_start.query()
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
