@@ -20,11 +20,13 @@
 //   warp 0       TMA producer: code tiles of A (128 rows) and W (256 rows) into a 4-stage ring
 //   warp 1       MMA issuer (owns the TMEM allocation): per stage, six tcgen05.cp of the
 //                stage's scale words from shared memory into its scale columns of TMEM,
-//                then four K = 64 MMAs (the copies and MMAs of one thread run in issue order)
-//   warps 4-7    scale producer: reads the tile rows' E8M0 words (16 bytes of a row, two
-//                stages, per load, two loads ahead) and stores each stage's words into a
-//                scale slot in shared memory (an 8-slot ring of its own) in the order
-//                tcgen05.cp reads them
+//                then four K = 64 MMAs (the copies and MMAs of one thread run in issue
+//                order) and one commit, which frees the stage's codes and scale slot; one
+//                wait per stage, on a barrier that takes the TMA bytes and the four scale
+//                warps' arrivals
+//   warps 4-7    scale producer: reads the tile rows' E8M0 words (32 bytes of a row, four
+//                stages, per load, two loads ahead) and stores each stage's words into the
+//                stage's scale slot in shared memory in the order tcgen05.cp reads them
 //   warps 8-11   epilogue: reads the float32 accumulator out of TMEM and stores C
 // Scale layout in TMEM (what the MMA reads): for a pair of K = 64 steps (four groups of
 // 32), row r of an operand with R rows has its four scale bytes in one 32-bit word at
@@ -72,9 +74,10 @@ static_assert(kColSf + kStages * kSfCols <= kTmemCols, "TMEM columns");
 constexpr int kSfBlockBytes = 512;
 constexpr int kSfSlotBytes = 6 * kSfBlockBytes;
 static_assert(kSfSlotBytes == (kBM + kBN) * 8, "8 scale bytes per row and stage");
-// The scale slots form their own ring, deeper than the code stages, so that the copies
-// (many small reads) have several stages of MMA time to land.
-constexpr int kSfStages = 8;
+// One scale slot per code stage: the stage's commit releases both, so the MMA thread issues
+// one commit per stage (a separate, deeper scale ring with its own commit measured slower:
+// the MMA thread's issue rate is what paces the pipe).
+constexpr int kSfStages = kStages;
 constexpr int kSfUnit = 4;  // stages of scale words per row read at once (32 bytes, one sector)
 constexpr int kOffSf = kStages * kStageBytes;
 constexpr int kSmem = kOffSf + kSfStages * kSfSlotBytes + 1024 /*barriers*/ + 1024 /*alignment*/;
@@ -82,15 +85,13 @@ static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 
 enum : uint32_t {
-  kStFull = 1u << 0, kStEmpty = 1u << 1, kStSfFull = 1u << 2, kStDFull = 1u << 3,
+  kStFull = 1u << 0, kStEmpty = 1u << 1, kStDFull = 1u << 3,
   kStDEmpty = 1u << 4, kStDrain = 1u << 5
 };
 
 struct Bars {
-  uint64_t full[kStages];     // TMA bytes of stage s landed
-  uint64_t empty[kStages];    // the MMAs that read stage s (codes and scale columns) completed
-  uint64_t sf_full[kSfStages];   // scale slot j filled (one arrive per scale warp)
-  uint64_t sf_empty[kSfStages];  // the copies out of scale slot j completed
+  uint64_t full[kStages];     // TMA bytes of stage s landed and its scale slot filled
+  uint64_t empty[kStages];    // the MMAs (and scale copies) that read stage s completed
   uint64_t d_full;            // accumulator of the tile complete
   uint64_t d_empty;           // accumulator read out (one arrive per epilogue warp)
   uint64_t mma_done;
@@ -268,12 +269,8 @@ mxgemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->full[s], 1 + 4);  // the producer's bytes and one arrive per scale warp
       mbar_init(&bars->empty[s], 1);
-    }
-    for (int j = 0; j < kSfStages; ++j) {
-      mbar_init(&bars->sf_full[j], 4);
-      mbar_init(&bars->sf_empty[j], 1);
     }
     mbar_init(&bars->d_full, 1);
     mbar_init(&bars->d_empty, 4);
@@ -339,8 +336,7 @@ mxgemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
       for (int kb = 0; kb < p.nk; ++kb, ++it) {
         const int s = it % kStages;
         const int j = it % kSfStages;
-        if (!warp_wait(&bars->full[s], (it / kStages) & 1, bars, p.status, kStFull) ||
-            !warp_wait(&bars->sf_full[j], (it / kSfStages) & 1, bars, p.status, kStSfFull)) {
+        if (!warp_wait(&bars->full[s], (it / kStages) & 1, bars, p.status, kStFull)) {
           ok = false;
           break;
         }
@@ -370,7 +366,6 @@ mxgemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
                      idesc_mxf4(id), sfa, sfb, (kb | k) != 0 ? 1u : 0u);
           }
           mma_commit_one(&bars->empty[s]);
-          mma_commit_one(&bars->sf_empty[j]);
         }
         __syncwarp();
       }
@@ -411,7 +406,7 @@ mxgemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
     auto put = [&](int it, const uint32_t (&w)[3][2]) {
       const int j = it % kSfStages;
       if (it >= kSfStages &&
-          !warp_wait(&bars->sf_empty[j], ((it / kSfStages) - 1) & 1, bars, p.status, kStEmpty)) {
+          !warp_wait(&bars->empty[j], ((it / kSfStages) - 1) & 1, bars, p.status, kStEmpty)) {
         ok = false;
         return;
       }
@@ -426,7 +421,7 @@ mxgemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__
         }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->sf_full[j]);
+      if (lane == 0) mbar_arrive(&bars->full[j]);
     };
     if (p.sf_vec) {
       // kSfUnit stages (8 kSfUnit bytes of a row) per load unit, issued two units ahead of
