@@ -139,3 +139,20 @@ def test_mx_matmul_rejects_bad_arguments():
         assert lib.fq_mx_matmul(T, O, L, p, p, p, p, vp(C.data_ptr()), vp(0), s) == _lib.FQ_ERR_INVALID
     assert lib.fq_mx_matmul(4, 4, 64, vp(buf.data_ptr() + 8), p, p, p, vp(C.data_ptr()), vp(0), s) \
         == _lib.FQ_ERR_INVALID
+
+
+def test_mx_matmul_full_size_sampled():
+    """The consumer contraction at the size bench.py times (T = 8192, O = 4096, L = 14336:
+    the row length of the 128x112 workload), operands drawn on the host; a sampled block of
+    C (random rows and columns plus the first, the last and those beside tile edges) against
+    the oracle's contraction of just those rows."""
+    T, O, L = 8192, 4096, 14336
+    rng = np.random.default_rng([T, O, L, 1])
+    a, sa = _operand(rng, T, L, lo=120, hi=133)
+    w, sw = _operand(rng, O, L, lo=120, hi=133)
+    C = _run(a, sa, w, sw, T, O, L)
+    ts = np.unique(np.concatenate([rng.choice(T, 20, replace=False), [0, 127, 128, T - 1]]))
+    os_ = np.unique(np.concatenate([rng.choice(O, 20, replace=False), [0, 255, 256, O - 1]]))
+    ref = oracle.mx_matmul(a[ts], sa[ts], w[os_], sw[os_], L)
+    worst = _check(C[np.ix_(ts, os_)], ref, _abs_ref(a[ts], sa[ts], w[os_], sw[os_], L), L)
+    print("full size sampled, worst/bound", worst)
