@@ -135,6 +135,9 @@ FQ_API fq_status fq_quantize_mx(fq_handle *h, const void *x, const void *P1, con
  *   w_fp4      [O, L/2] bytes, 16-byte aligned; w_scale_e8m0 [O, ceilDiv(L, 64), 2] bytes
  *   C          [T, O] float32, row-major (4-byte aligned; O % 4 == 0 with a 16-byte aligned C
  *              takes the vector stores)
+ *   (the scale arrays need no alignment; 16-byte aligned ones whose row stride
+ *   2 * ceilDiv(L, 64) is a multiple of 16 bytes are read 16 bytes at a time, others word
+ *   by word)
  *   status     a device word, or NULL: a bounded wait that gives up ORs a nonzero code into
  *              it and leaves C undefined (with NULL nothing reports that)
  * Allocates nothing; asynchronous on stream. Errors: FQ_ERR_NULLPTR (a_fp4, a_scale_e8m0,
