@@ -74,9 +74,10 @@ struct Geo {
   static_assert(N % 16 == 0 && N >= 64 && N <= 128, "tensor-core kernel covers N in [64,128], N % 16 == 0");
   static constexpr int kAtoms = (N + 63) / 64;              // 64-element swizzle atoms along N
   static constexpr int kXStage = kAtoms * 128 * 128;        // bytes per x stage
-  // x ring depth: five stages at N = 80 .. 112 (2-3 % faster than four at 128 x 112),
-  // four at N = 64 (eight measured slower: the longer first round of loads delays the
-  // first tile), three at N = 128 where BD(P1) stays in shared memory
+  // x ring depth: five stages at N = 80 .. 112 (two to five measure within noise of one
+  // another at 128 x 112: the loads land well ahead), four at N = 64 (eight measured
+  // slower: the longer first round of loads delays the first tile), three at N = 128
+  // where BD(P1) stays in shared memory
   static constexpr int kStages = N == 128 ? 3 : (N == 64 ? 4 : 5);
   // BD(P1) sits in TMEM (64 columns; stage A is then a TS MMA that reads only the x tile
   // from shared memory, 3.5 KB instead of 7.5 KB per MMA at N = 112) when four N-column
