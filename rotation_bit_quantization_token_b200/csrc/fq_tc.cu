@@ -538,16 +538,23 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
     }
   } else if (!G::kP1Tmem && tid < 256) {
     // BD(P1): 128 x 128, K-major, 128B swizzle; element (r, k) = P1[r % M][k % M] on the
-    // diagonal blocks (r / M == k / M), else 0.
+    // diagonal blocks (r / M == k / M), else 0. All eight loads first, then the stores: a
+    // store between them would keep the compiler from issuing the next load (it cannot
+    // tell the two pointers apart), one round trip each.
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       const int c = tid + 256 * q;
       const int r = c >> 4, kc = c & 15, k = kc * 8;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (r / M == k / M)
-        v = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.P1) + (r % M) * M + (k % M));
+      buf[q] = r / M == k / M
+                   ? *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.P1) + (r % M) * M + (k % M))
+                   : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int c = tid + 256 * q;
+      const int r = c >> 4, kc = c & 15;
       const uint32_t off = G::kOffP1 + (kc >> 3) * 16384 + r * 128 + ((((kc & 7) ^ (r & 7))) << 4);
-      *reinterpret_cast<uint4*>(smem + off) = v;
+      *reinterpret_cast<uint4*>(smem + off) = buf[q];
     }
   }
   float lmax = 0.0f;
