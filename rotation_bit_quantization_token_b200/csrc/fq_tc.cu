@@ -354,12 +354,6 @@ __device__ __forceinline__ float absmax16(const float* v) {
   const float e = max3abs(v[12], v[13], v[14]);
   return fmaxf(max3abs(a, b, c), max3abs(d, e, v[15]));
 }
-// insert the low 4 bits of src into acc at bit position pos
-__device__ __forceinline__ uint32_t bfi4(uint32_t src, uint32_t acc, int pos) {
-  uint32_t r;
-  asm("bfi.b32 %0, %1, %2, %3, 4;" : "=r"(r) : "r"(src), "r"(acc), "r"(pos));
-  return r;
-}
 // eight E2M1 codes (round to nearest even, saturate) in one word: element 0 in bits 0-3
 __device__ __forceinline__ uint32_t e2m1x8(float2 a, float2 b, float2 c, float2 d) {
   uint32_t r;
@@ -871,17 +865,15 @@ tc_kernel(const __grid_constant__ CUtensorMap tmap, const TcParams p) {
             for (int wd = 0; wd < 2; ++wd) {
               const float* w = d + c * 16 + wd * 8;
               if constexpr (kMode == kModePerToken) {
-                const float2 magic = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+                // integer nearest (ties to even), then clamped to [-8, 7] and packed by the
+                // saturating pack: it puts its second operand in the low nibble, its first
+                // above it, and the carried word above both, so the highest pair goes first
                 uint32_t acc = 0u;
 #pragma unroll
-                for (int e = 0; e < 8; e += 2) {
-                  float2 t = __fmul2_rn(make_float2(w[e], w[e + 1]), F2);
-                  t.x = fminf(fmaxf(t.x, -8.0f), 7.0f);
-                  t.y = fminf(fmaxf(t.y, -8.0f), 7.0f);
-                  // adding 1.5 * 2^23 rounds to an integer (half to even) held in the low bits
-                  const float2 u = __fadd2_rn(t, magic);
-                  acc = bfi4(__float_as_uint(u.x), acc, 4 * e);
-                  acc = bfi4(__float_as_uint(u.y), acc, 4 * e + 4);
+                for (int e = 6; e >= 0; e -= 2) {
+                  const float2 t = __fmul2_rn(make_float2(w[e], w[e + 1]), F2);
+                  const int lo = __float2int_rn(t.x), hi = __float2int_rn(t.y);
+                  asm("cvt.pack.sat.s4.s32.b32 %0, %1, %2, %3;" : "=r"(acc) : "r"(hi), "r"(lo), "r"(acc));
                 }
                 words[wd] = acc;
               } else {
