@@ -75,8 +75,9 @@ constexpr int kSfBlockBytes = 512;
 constexpr int kSfSlotBytes = 6 * kSfBlockBytes;
 static_assert(kSfSlotBytes == (kBM + kBN) * 8, "8 scale bytes per row and stage");
 // One scale slot per code stage: the stage's commit releases both, so the MMA thread issues
-// one commit per stage (a separate, deeper scale ring with its own commit measured slower:
-// the MMA thread's issue rate is what paces the pipe).
+// one commit and waits once per stage (a separate, deeper scale ring with its own commit and
+// barrier measured 5-10 % slower: the barrier round trips in the MMA thread's loop pace the
+// pipe, not its instruction count).
 constexpr int kSfStages = kStages;
 constexpr int kSfUnit = 4;  // stages of scale words per row read at once (32 bytes, one sector)
 constexpr int kOffSf = kStages * kStageBytes;
