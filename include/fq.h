@@ -110,7 +110,7 @@ FQ_API fq_status fq_quantize_per_token(fq_handle *h, const void *x, const void *
  *   dstTypeMax 0.0 (case 1), 6.0 or 7.0 (case 2), any other value in [6, 12] (case 3)
  *   out_fp4    [K, M*N] E2M1 codes, two per byte: K*M*N/2 bytes
  *   scale_e8m0 [K, ceilDiv(M*N, 64), 2] E8M0 bytes; group g of token k at byte
- *              k*2*ceilDiv(M*N,64) + g; the pad byte of an odd group count is 0x00
+ *              k*2*ceilDiv(M*N,64) + g; the spare byte of an odd group count is 0x7F (2^0)
  * Errors: FQ_ERR_NULLPTR (h, x, P1, out_fp4, scale_e8m0), FQ_ERR_INVALID (dstTypeMax
  * outside {0} U [6, 12], N odd, misaligned pointer), FQ_ERR_CUDA. */
 FQ_API fq_status fq_quantize_mx(fq_handle *h, const void *x, const void *P1, const void *P2,

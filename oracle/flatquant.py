@@ -37,7 +37,8 @@ Readings taken where the page is silent or garbled:
   value whose magnitude rounds to zero encodes as +0 (0x0), so the format's two zero
   codes never both appear (the page gives no rule for the sign of a zero code, and a
   sign kept on values that round to zero would hinge on the last bit of x'').
-* The pad byte of an odd group count is the scale of a group of 32 zeros (0x00).
+* The spare byte of an odd group count (the scale tensor holds ceilDiv(M*N, 64) pairs) is
+  0x7F, the scale 2^0: the page gives it no value.
 """
 
 import numpy as np
@@ -309,11 +310,10 @@ def mx_quantize(x2, dst_type_max):
 
 def mx_scale_layout(group_bytes):
     """Place per-group E8M0 bytes in the page's [K, ceilDiv(M*N, 64), 2] scale tensor
-    (group g at [k, g // 2, g % 2]); the pad slot of an odd group count holds the scale
-    of an all-zero group (0x00)."""
+    (group g at [k, g // 2, g % 2]); the spare slot of an odd group count holds 0x7F (2^0)."""
     group_bytes = np.asarray(group_bytes, dtype=np.uint8)
     K, G = group_bytes.shape
-    out = np.zeros((K, -(-G // 2) * 2), dtype=np.uint8)
+    out = np.full((K, -(-G // 2) * 2), 0x7F, dtype=np.uint8)
     out[:, :G] = group_bytes
     return out.reshape(K, -1, 2)
 

@@ -152,9 +152,9 @@ general_kernel(const GeneralParams p) {
         }
         __syncthreads();
       } else if (pass == 0 && p.mode == kModeMx) {
-        const int gs = 2 * ((MN + 63) / 64);  // scale bytes per token, with the pad slot
+        const int gs = 2 * ((MN + 63) / 64);  // scale bytes per token, with the spare slot
         for (int g = tid; g < gs; g += kThreads) {
-          uint32_t byte = 0u;
+          uint32_t byte = 0x7Fu;  // the spare slot of an odd group count: 2^0
           if (g < G) {
             const MxScale s = mx_scale(__uint_as_float(gmax[g]), p.rule);
             byte = s.byte;

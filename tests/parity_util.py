@@ -112,9 +112,9 @@ def compare_mx(out_bytes, scales, ref_info, D, elem_taint=None):
     got = unpack_nibbles(np.asarray(out_bytes).reshape(K, -1))[:, :L]
     got_b = np.asarray(scales).reshape(K, -1)
     want_b = ref_info["group_bytes"]
-    # the pad slot of an odd group count is 0x00
+    # the spare slot of an odd group count is 0x7F (2^0)
     if got_b.shape[1] > G:
-        assert np.all(got_b[:, G:] == 0), "pad scale byte is not 0x00"
+        assert np.all(got_b[:, G:] == 0x7F), "spare scale byte is not 0x7F"
     got_b = got_b[:, :G].astype(np.int64)
     gex = group_exempt(ref_info["amax"], D)
     if elem_taint is not None:

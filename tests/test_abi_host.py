@@ -243,5 +243,5 @@ def test_output_buffer_checks_on_host():
     for t, nbytes, dtype, word in bad:
         with pytest.raises((ValueError, TypeError), match=word):
             api._check_output("buf", t, nbytes, cpu, dtype)
-    # scale tensor of an odd group count: [K, ceilDiv(M*N, 64), 2] includes the pad slot
+    # scale tensor of an odd group count: [K, ceilDiv(M*N, 64), 2] includes the spare slot
     assert api._scale_bytes(2, 3, 32) == 2 * 2 * 2

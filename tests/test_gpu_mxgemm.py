@@ -26,12 +26,12 @@ pytestmark = pytest.mark.gpu
 
 
 def _operand(rng, rows, L, lo=118, hi=136):
-    """Random packed E2M1 codes [rows, L/2] and scale bytes [rows, ceilDiv(L, 64), 2]; the pad
-    slot of an odd group count is 0x00, as the operator writes it."""
+    """Random packed E2M1 codes [rows, L/2] and scale bytes [rows, ceilDiv(L, 64), 2]; the spare
+    slot of an odd group count is 0x7F, as the operator writes it."""
     codes = rng.integers(0, 256, size=(rows, L // 2), dtype=np.uint8)
     G = L // 32
     S = -(-L // 64)
-    sc = np.zeros((rows, 2 * S), dtype=np.uint8)
+    sc = np.full((rows, 2 * S), 0x7F, dtype=np.uint8)
     sc[:, :G] = rng.integers(lo, hi + 1, size=(rows, G), dtype=np.uint8)
     return codes, sc.reshape(rows, S, 2)
 

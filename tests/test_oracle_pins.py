@@ -319,7 +319,7 @@ def test_mx_power_of_two_shift_invariance():
 def test_mx_groups_straddle_rows_and_pad():
     """Groups run over the flattened [K, M*N] axis, across row ends (N = 112 gives 3.5
     groups per row), and a short last group is zero padded; the scale tensor is
-    [K, ceilDiv(M*N, 64), 2] with the odd slot holding the all-zero-group byte."""
+    [K, ceilDiv(M*N, 64), 2] with the spare slot of an odd group count holding 0x7F (2^0)."""
     rng = _rng(36)
     x2 = rng.standard_normal((2, 3, 14))  # M*N = 42: one full group + a group of 10
     codes, gbytes, v, amax = oracle.mx_quantize(x2, 0.0)
@@ -331,7 +331,7 @@ def test_mx_groups_straddle_rows_and_pad():
     x3 = rng.standard_normal((2, 1, 96))  # three groups -> ceilDiv(96, 64) = 2 -> pad slot
     _, gb3, _, _ = oracle.mx_quantize(x3, 0.0)
     sc3 = oracle.mx_scale_layout(gb3)
-    assert sc3.shape == (2, 2, 2) and np.all(sc3[:, 1, 1] == 0)
+    assert sc3.shape == (2, 2, 2) and np.all(sc3[:, 1, 1] == 0x7F)
     assert np.array_equal(sc3.reshape(2, -1)[:, :3], gb3)
 
 
