@@ -133,6 +133,25 @@ def test_edge_shapes(shape, mode):
         _run_and_compare(w, x, P1, P2, kernel)
 
 
+@pytest.mark.parametrize("shape", [(741, 128, 80), (741, 128, 96), (1481, 64, 80),
+                                   (2963, 32, 96), (1481, 64, 128)])
+@pytest.mark.parametrize("mode", ["per_token", "mx6", "mx10"])
+def test_multi_tile_other_widths(shape, mode):
+    """The tensor-core widths no workload uses (N = 80, 96; M = 32 packing; N = 128 at
+    M = 64), at about five 128-row tiles per SM plus a ragged tail, so every TMEM slot and
+    ring stage is reused several times and, at N = 96, both stage-B issuer warps run."""
+    K, M, N = shape
+    from rotation_bit_quantization_token_b200.workloads import Workload
+    if mode == "per_token":
+        w = Workload("multi", K, M, N, "per_token", "normal", out="int4", clip_ratio=0.9)
+    else:
+        w = Workload("multi", K, M, N, "mx", "normal_outliers", dst_type_max=float(mode[2:]))
+    x, P1, P2 = make_inputs(w, seed=K + M + N)
+    kernels = _kernels_for(w)
+    assert "tcgen05" in kernels
+    _run_and_compare(w, x, P1, P2, "tcgen05")
+
+
 @pytest.mark.parametrize("shape", [(5, 128, 112), (7, 64, 64), (3, 32, 96)])
 @pytest.mark.parametrize("mode", ["per_token", "mx10"])
 def test_fp16_inputs_tensor_core_shapes(shape, mode):
