@@ -86,7 +86,7 @@ def compare_per_token(out_bytes, qs, ref_codes, ref_qs, ref_v, elem_taint=None, 
     assert np.all(np.abs(got - want)[diff] <= 1), "exempt INT4 codes differ by more than one"
     assert stats["mismatch"] <= MAX_MISMATCH_FRAC * want.size, stats
     # quantScale within 1e-6 relative (about 8 ulp) of the reference: it is the maximum of
-    # the kernel's float32 x'', which carries the accumulation's rounding (up to 5 ulp seen).
+    # the kernel's float32 x'', which carries the accumulation's rounding (up to 7 ulp seen).
     # For non-negative floats the difference of the bit patterns counts the ulps between them.
     qs32 = np.asarray(qs, dtype=np.float32).reshape(-1)
     rq32 = np.asarray(ref_qs, dtype=np.float32).reshape(-1)
